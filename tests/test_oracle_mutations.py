@@ -1,0 +1,70 @@
+"""Mutation check of the oracle pins: plant one plausible mistake at a time in
+a copy of oracle.c (on the CPU, in a temporary directory), rebuild it, and
+assert that at least one pin fails.  A pin set that let a planted mistake
+through would not be pinning the oracle."""
+import os
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+SRC = os.path.join(os.path.dirname(oracle.__file__), "oracle.c")
+
+MUTATIONS = {
+    "alibi_sign": ("val += -slopes[h] * fabs((double)(i - j));",
+                   "val += slopes[h] * fabs((double)(i - j));"),
+    "causal_strict": ("if (m->causal && j > i) return 0;",
+                      "if (m->causal && j >= i) return 0;"),
+    "padding_off_by_one": ("if (m->kv_len && j >= m->kv_len[b]) return 0;",
+                           "if (m->kv_len && j > m->kv_len[b]) return 0;"),
+    "lse_without_max": ("lse[i] = mx + log(sum);", "lse[i] = log(sum);"),
+    "dk_without_scale": ("dkh[(int64_t)j * D + d] = scale * acc;",
+                         "dkh[(int64_t)j * D + d] = acc;"),
+    "ds_sign": ("ds[(int64_t)i * Sk + j] = pij * (ds[(int64_t)i * Sk + j] - dl);",
+                "ds[(int64_t)i * Sk + j] = pij * (dl - ds[(int64_t)i * Sk + j]);"),
+    "modality_transposed": ("else if (a == 0 && c == 1) ok = m->allow01;",
+                            "else if (a == 0 && c == 1) ok = m->allow10;"),
+    "dq_uses_q": ("acc += ds[(int64_t)i * Sk + j] * kh[(int64_t)j * D + d];",
+                  "acc += ds[(int64_t)i * Sk + j] * qh[(int64_t)j * D + d];"),
+}
+
+CHECKS = [
+    lambda: pins.test_hand_two_keys("none"),
+    lambda: pins.test_hand_two_keys("causal"),
+    pins.test_alibi_q0_closed_form,
+    lambda: pins.test_q_zero_gives_mean_of_allowed_v("padding"),
+    lambda: pins.test_q_zero_gives_mean_of_allowed_v("modality"),
+    lambda: pins.test_matches_torch_sdpa_fwd_bwd("causal", (13, 13)),
+    lambda: pins.test_matches_torch_sdpa_fwd_bwd("padding", (7, 19)),
+    lambda: pins.test_bwd_finite_differences("none", True),
+]
+
+
+def _any_check_fails():
+    for chk in CHECKS:
+        try:
+            chk()
+        except (AssertionError, RuntimeError):
+            return True
+    return False
+
+
+@pytest.mark.parametrize("name", sorted(MUTATIONS))
+def test_planted_mistake_is_caught(name, tmp_path):
+    before, after = MUTATIONS[name]
+    src = open(SRC).read()
+    assert src.count(before) == 1, f"mutation anchor for {name} not found once"
+    mutated = tmp_path / "oracle_mut.c"
+    mutated.write_text(src.replace(before, after))
+    so = tmp_path / "liboracle_mut.so"
+    subprocess.run(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-std=c11",
+                    "-o", str(so), str(mutated), "-lm"], check=True)
+    with oracle.use_library(str(so)):
+        assert _any_check_fails(), f"planted mistake '{name}' passed every pin"
+
+
+def test_unmutated_oracle_passes_the_same_checks():
+    assert not _any_check_fails()
