@@ -1,0 +1,284 @@
+// abi.cu -- the extern "C" entry points declared in include/fa.h: argument
+// validation on the host, problem set-up, and dispatch to the launchers.
+//
+// The call follows npu_fusion_attention of the FlashAttentionScore guide
+// (sec. 3.1 call, sec. 3.2 parameter table): query/key/value, head count,
+// input layout BNSD or BSH, optional pse (ALiBi here), attention mask
+// (causal, key padding, bool, modality rule), scale and keep_prob (1.0 only).
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "../../include/fa.h"
+#include "fa_common.cuh"
+#include "launch.h"
+
+namespace fa {
+// Device status word: kernels OR bit 0 into it when a bounded wait gives up.
+__device__ unsigned int g_fa_status = 0;
+}  // namespace fa
+
+namespace {
+
+using fa::Problem;
+
+constexpr int kMaxModalityKeys = 32768;
+
+bool aligned16(const void* ptr) {
+  return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0;
+}
+
+fa_status check_shape(const fa_shape* s) {
+  if (!s) return FA_ERR_INVALID_ARG;
+  if (s->B < 0 || s->N < 0 || s->Sq < 0 || s->Sk < 0 || s->D <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (s->layout != FA_LAYOUT_BNSD && s->layout != FA_LAYOUT_BSH)
+    return FA_ERR_INVALID_ARG;
+  if (s->dtype != FA_F32 && s->dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (s->dtype == FA_BF16 && s->D != 64 && s->D != 128) return FA_ERR_UNSUPPORTED;
+  if (s->dtype == FA_F32 && s->D > 128) return FA_ERR_UNSUPPORTED;
+  if (s->B > 65535 || s->N > 65535) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+// Fills the kernel-side problem from the ABI arguments (after validation).
+fa_status make_problem(const fa_shape* s, const fa_pse* pse, const fa_mask* m,
+                       float scale, float keep_prob, Problem* p) {
+  fa_status st = check_shape(s);
+  if (st != FA_OK) return st;
+  if (!isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (!(keep_prob == 1.0f)) return FA_ERR_UNSUPPORTED;
+  Problem q = {};
+  q.B = s->B;
+  q.N = s->N;
+  q.Sq = s->Sq;
+  q.Sk = s->Sk;
+  q.D = s->D;
+  q.layout = s->layout;
+  const int64_t H = int64_t(s->N) * s->D;
+  if (s->layout == FA_LAYOUT_BNSD) {
+    q.q_sb = int64_t(s->N) * s->Sq * s->D;
+    q.q_sh = int64_t(s->Sq) * s->D;
+    q.q_ss = s->D;
+    q.k_sb = int64_t(s->N) * s->Sk * s->D;
+    q.k_sh = int64_t(s->Sk) * s->D;
+    q.k_ss = s->D;
+  } else {
+    q.q_sb = int64_t(s->Sq) * H;
+    q.q_sh = s->D;
+    q.q_ss = H;
+    q.k_sb = int64_t(s->Sk) * H;
+    q.k_sh = s->D;
+    q.k_ss = H;
+  }
+  q.scale = scale;
+  q.scale_log2 = scale * fa::kLog2e;
+  q.tm_heads = 1;
+  if (m) {
+    const uint32_t known = FA_MASK_CAUSAL | FA_MASK_KV_PADDING | FA_MASK_BOOL |
+                           FA_MASK_MODALITY;
+    if (m->flags & ~known) return FA_ERR_INVALID_ARG;
+    q.mask_flags = m->flags;
+    if (m->flags & FA_MASK_KV_PADDING) {
+      if (!m->kv_len) return FA_ERR_INVALID_ARG;
+      q.kv_len = m->kv_len;
+    }
+    if (m->flags & FA_MASK_BOOL) {
+      if (!m->mask) return FA_ERR_INVALID_ARG;
+      if (m->mask_stride_b < 0 || m->mask_stride_h < 0 || m->mask_stride_q < 0)
+        return FA_ERR_INVALID_ARG;
+      q.mask = m->mask;
+      q.m_sb = m->mask_stride_b;
+      q.m_sh = m->mask_stride_h;
+      q.m_sq = m->mask_stride_q;
+      q.tile_map = m->tile_map;
+      q.tm_heads = m->mask_stride_h == 0 ? 1 : s->N;
+    }
+    if (m->flags & FA_MASK_MODALITY) {
+      if (!m->modality_ids) return FA_ERR_INVALID_ARG;
+      if (s->Sq != s->Sk) return FA_ERR_INVALID_ARG;
+      if (s->Sk > kMaxModalityKeys) return FA_ERR_UNSUPPORTED;
+      q.ids = m->modality_ids;
+      q.allow_bits = (m->allow[0][0] ? 1u : 0u) | (m->allow[0][1] ? 2u : 0u) |
+                     (m->allow[1][0] ? 4u : 0u) | (m->allow[1][1] ? 8u : 0u) |
+                     (m->allow_diag ? 16u : 0u);
+    }
+  }
+  if (pse) {
+    if (pse->kind == FA_PSE_ALIBI) {
+      if (!pse->slopes) return FA_ERR_INVALID_ARG;
+      q.slopes = pse->slopes;
+    } else if (pse->kind != FA_PSE_NONE) {
+      return FA_ERR_INVALID_ARG;
+    }
+  }
+  *p = q;
+  return FA_OK;
+}
+
+// Device address of g_fa_status on the current device (looked up once per
+// device; the symbol lives in every device's copy of the module).
+unsigned int* status_word() {
+  static unsigned int* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, fa::g_fa_status) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<unsigned int*>(a);
+  }
+  return addr[dev];
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+size_t elem_size(const fa_shape* s) { return s->dtype == FA_BF16 ? 2 : 4; }
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+  }
+  return "FA_ERR_UNKNOWN";
+}
+
+const char* fa_version(void) { return "fa_b200 1.0 sm_100a"; }
+
+fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
+                 const void* v, const fa_pse* pse, const fa_mask* mask,
+                 float scale, float keep_prob, void* out, float* lse,
+                 void* stream) {
+  Problem p;
+  fa_status st = make_problem(shape, pse, mask, scale, keep_prob, &p);
+  if (st != FA_OK) return st;
+  if (p.B == 0 || p.N == 0 || p.Sq == 0) return FA_OK;  // nothing to write
+  p.status = status_word();
+  if (!p.status) return FA_ERR_CUDA;
+  if (!q || !out || !lse || (p.Sk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(out) || (p.Sk > 0 && (!aligned16(k) || !aligned16(v))) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_INVALID_ARG;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const bool bf16 = shape->dtype == FA_BF16;
+  cudaError_t e;
+  if (p.Sk == 0)
+    e = fa::launch_fill_empty_rows(p, bf16, out, lse, cs);
+  else if (bf16)
+    e = fa::launch_fwd_bf16_sm100(p, q, k, v, out, lse, cs);
+  else
+    e = fa::launch_fwd_f32(p, q, k, v, out, lse, cs);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(const fa_shape* shape) {
+  if (check_shape(shape) != FA_OK) return 0;
+  const size_t rows = size_t(shape->B) * shape->N * shape->Sq;
+  return round_up(rows * shape->D * sizeof(float), 256) +
+         round_up(rows * sizeof(float), 256);
+}
+
+fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
+                 const void* v, const void* out, const void* dout,
+                 const float* lse, const fa_pse* pse, const fa_mask* mask,
+                 float scale, float keep_prob, void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  Problem p;
+  fa_status st = make_problem(shape, pse, mask, scale, keep_prob, &p);
+  if (st != FA_OK) return st;
+  if (p.B == 0 || p.N == 0) return FA_OK;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const size_t es = elem_size(shape);
+  if (p.Sq == 0 || p.Sk == 0) {
+    // No (query, key) pair: every gradient is zero.
+    if (p.Sq == 0 && p.Sk > 0) {
+      if (!dk || !dv) return FA_ERR_INVALID_ARG;
+      const size_t n = size_t(p.B) * p.N * p.Sk * p.D * es;
+      if (cudaMemsetAsync(dk, 0, n, cs) != cudaSuccess ||
+          cudaMemsetAsync(dv, 0, n, cs) != cudaSuccess)
+        return FA_ERR_CUDA;
+    }
+    if (p.Sk == 0 && p.Sq > 0) {
+      if (!dq) return FA_ERR_INVALID_ARG;
+      const size_t n = size_t(p.B) * p.N * p.Sq * p.D * es;
+      if (cudaMemsetAsync(dq, 0, n, cs) != cudaSuccess) return FA_ERR_CUDA;
+    }
+    return FA_OK;
+  }
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv || !workspace)
+    return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(dout) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      !aligned16(workspace) || (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_size(shape)) return FA_ERR_INVALID_ARG;
+  p.status = status_word();
+  if (!p.status) return FA_ERR_CUDA;
+  const size_t rows = size_t(p.B) * p.N * p.Sq;
+  float* dq_acc = static_cast<float*>(workspace);
+  float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                          round_up(rows * p.D * sizeof(float), 256));
+  const bool bf16 = shape->dtype == FA_BF16;
+  cudaError_t e = fa::launch_bwd_pre(p, bf16, out, dout, delta, dq_acc, cs);
+  if (e == cudaSuccess) {
+    if (bf16)
+      e = fa::launch_bwd_bf16_sm100(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, cs);
+    else
+      e = fa::launch_bwd_f32(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, cs);
+  }
+  if (e == cudaSuccess) e = fa::launch_bwd_post(p, bf16, dq_acc, dq, cs);
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_mask_tile_map_size(const fa_shape* shape, const fa_mask* mask) {
+  if (check_shape(shape) != FA_OK || !mask || !(mask->flags & FA_MASK_BOOL))
+    return 0;
+  const size_t heads = mask->mask_stride_h == 0 ? 1 : size_t(shape->N);
+  const size_t nqt = (size_t(shape->Sq) + FA_TILE_M - 1) / FA_TILE_M;
+  const size_t nkt = (size_t(shape->Sk) + FA_TILE_N - 1) / FA_TILE_N;
+  return size_t(shape->B) * heads * nqt * nkt;
+}
+
+fa_status fa_build_mask_tile_map(const fa_shape* shape, const fa_mask* mask,
+                                 uint8_t* tile_map, void* stream) {
+  Problem p;
+  fa_status st = make_problem(shape, nullptr, mask, 1.0f, 1.0f, &p);
+  if (st != FA_OK) return st;
+  if (!mask || !(mask->flags & FA_MASK_BOOL) || !tile_map) return FA_ERR_INVALID_ARG;
+  cudaError_t e = fa::launch_tile_map(p, tile_map, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_build_modality_mask(int B, int S, const int32_t* modality_ids,
+                                 const uint8_t allow[2][2], int allow_diag,
+                                 uint8_t* mask_out, void* stream) {
+  if (B < 0 || S < 0 || !allow) return FA_ERR_INVALID_ARG;
+  if (B == 0 || S == 0) return FA_OK;
+  if (!modality_ids || !mask_out) return FA_ERR_INVALID_ARG;
+  const uint32_t bits = (allow[0][0] ? 1u : 0u) | (allow[0][1] ? 2u : 0u) |
+                        (allow[1][0] ? 4u : 0u) | (allow[1][1] ? 8u : 0u) |
+                        (allow_diag ? 16u : 0u);
+  cudaError_t e = fa::launch_modality_mask(B, S, modality_ids, bits, mask_out,
+                                           static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_sync_status(void* stream) {
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, fa::g_fa_status, sizeof(word)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (word != 0 &&
+      cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(zero)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return word ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+}  // extern "C"

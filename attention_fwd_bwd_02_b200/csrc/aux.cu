@@ -1,0 +1,197 @@
+// aux.cu -- the small HBM-bound kernels around the attention main loops:
+//   * bwd_pre : Delta_i = sum_d dO_id * O_id (fp32) and zeroing of the fp32
+//               dQ accumulator;
+//   * bwd_post: dQ = scale * dQacc, cast to the tensor dtype and layout;
+//   * tile_map: classification of 128 x 128 tiles of a bool mask;
+//   * modality_mask: the explicit cross-modal bool mask from modality ids
+//     (create_cross_modal_mask of the multimodal FlashAttention page,
+//     layer 2, with a 2x2 allow table).
+// All are grid-strided, 16-byte vectorised where the layout allows.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "fa_common.cuh"
+#include "launch.h"
+
+namespace fa {
+
+namespace {
+
+__device__ __forceinline__ float to_f(float x) { return x; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+__device__ __forceinline__ void from_f(float v, float* dst) { *dst = v; }
+__device__ __forceinline__ void from_f(float v, __nv_bfloat16* dst) {
+  *dst = __float2bfloat16_rn(v);
+}
+
+// One warp per query row: Delta = dot(dO_i, O_i).  Also clears the row of the
+// dQ accumulator ([B][N][Sq][D] fp32).
+template <typename T>
+__global__ void bwd_pre_kernel(Problem p, const T* __restrict__ out,
+                               const T* __restrict__ dout,
+                               float* __restrict__ delta,
+                               float* __restrict__ dq_acc) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       r < rows; r += warps) {
+    const int i = int(r % p.Sq);
+    const int64_t bh = r / p.Sq;
+    const int h = int(bh % p.N), b = int(bh / p.N);
+    const int64_t off = b * p.q_sb + h * p.q_sh + int64_t(i) * p.q_ss;
+    float acc = 0.f;
+    for (int d = lane; d < p.D; d += 32)
+      acc = fmaf(to_f(dout[off + d]), to_f(out[off + d]), acc);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(~0u, acc, o);
+    if (lane == 0) delta[r] = acc;
+    float* z = dq_acc + r * p.D;
+    for (int d = lane; d < p.D; d += 32) z[d] = 0.f;
+  }
+}
+
+template <typename T>
+__global__ void bwd_post_kernel(Problem p, const float* __restrict__ dq_acc,
+                                T* __restrict__ dq) {
+  const int64_t total = int64_t(p.B) * p.N * p.Sq * p.D;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int d = int(e % p.D);
+    const int64_t r = e / p.D;
+    const int i = int(r % p.Sq);
+    const int64_t bh = r / p.Sq;
+    const int h = int(bh % p.N), b = int(bh / p.N);
+    from_f(dq_acc[e] * p.scale,
+           dq + b * p.q_sb + h * p.q_sh + int64_t(i) * p.q_ss + d);
+  }
+}
+
+// One CTA per tile: 256 threads scan the 128 x 128 bytes of the mask tile.
+__global__ void tile_map_kernel(Problem p, uint8_t* __restrict__ tile_map) {
+  const int nqt = (p.Sq + FA_TILE_M - 1) / FA_TILE_M;
+  const int nkt = (p.Sk + FA_TILE_N - 1) / FA_TILE_N;
+  const int64_t t = blockIdx.x;
+  const int kt = int(t % nkt);
+  const int qt = int((t / nkt) % nqt);
+  const int64_t bh = t / (int64_t(nkt) * nqt);
+  const int h = int(bh % p.tm_heads), b = int(bh / p.tm_heads);
+  const int i0 = qt * FA_TILE_M, j0 = kt * FA_TILE_N;
+  const int rows = min(FA_TILE_M, p.Sq - i0), cols = min(FA_TILE_N, p.Sk - j0);
+  int any = 0, all = 1;
+  for (int e = threadIdx.x; e < rows * cols; e += blockDim.x) {
+    const int r = e / cols, c = e % cols;
+    const uint8_t m = p.mask[b * p.m_sb + h * p.m_sh + int64_t(i0 + r) * p.m_sq + j0 + c];
+    any |= (m != 0);
+    all &= (m != 0);
+  }
+  any = __syncthreads_or(any);
+  all = __syncthreads_and(all);
+  if (threadIdx.x == 0) tile_map[t] = any ? (all ? 2 : 1) : 0;
+}
+
+__global__ void modality_mask_kernel(int B, int S, const int32_t* __restrict__ ids,
+                                     uint32_t allow_bits, uint8_t* __restrict__ mask) {
+  const int64_t total = int64_t(B) * S * S;
+  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
+       e += int64_t(gridDim.x) * blockDim.x) {
+    const int j = int(e % S);
+    const int64_t r = e / S;
+    const int i = int(r % S), b = int(r / S);
+    mask[e] = modality_ok(allow_bits, ids[int64_t(b) * S + i],
+                          ids[int64_t(b) * S + j], i, j)
+                  ? 1
+                  : 0;
+  }
+}
+
+// Rows with no visible key at all (Sk == 0): out = 0, lse = -inf.
+template <typename T>
+__global__ void fill_empty_kernel(Problem p, T* __restrict__ out,
+                                  float* __restrict__ lse) {
+  const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  for (int64_t r = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; r < rows;
+       r += int64_t(gridDim.x) * blockDim.x) {
+    const int i = int(r % p.Sq);
+    const int64_t bh = r / p.Sq;
+    const int h = int(bh % p.N), b = int(bh / p.N);
+    T* o = out + b * p.q_sb + h * p.q_sh + int64_t(i) * p.q_ss;
+    for (int d = 0; d < p.D; ++d) from_f(0.f, o + d);
+    lse[r] = -INFINITY;
+  }
+}
+
+int grid_for(int64_t work, int per_block) {
+  int64_t g = (work + per_block - 1) / per_block;
+  const int64_t cap = 148 * 16;  // a few waves of the 148 SMs is plenty
+  if (g > cap) g = cap;
+  return g < 1 ? 1 : int(g);
+}
+
+}  // namespace
+
+cudaError_t launch_fill_empty_rows(const Problem& p, bool is_bf16, void* out,
+                                   float* lse, cudaStream_t st) {
+  const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  const int g = grid_for(rows, 256);
+  if (is_bf16)
+    fill_empty_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+        p, static_cast<__nv_bfloat16*>(out), lse);
+  else
+    fill_empty_kernel<float><<<g, 256, 0, st>>>(p, static_cast<float*>(out), lse);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_pre(const Problem& p, bool is_bf16, const void* out,
+                           const void* dout, float* delta, float* dq_acc,
+                           cudaStream_t st) {
+  const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  const int g = grid_for(rows, 8);
+  if (is_bf16)
+    bwd_pre_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+        p, static_cast<const __nv_bfloat16*>(out),
+        static_cast<const __nv_bfloat16*>(dout), delta, dq_acc);
+  else
+    bwd_pre_kernel<float><<<g, 256, 0, st>>>(
+        p, static_cast<const float*>(out), static_cast<const float*>(dout),
+        delta, dq_acc);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_post(const Problem& p, bool is_bf16,
+                            const float* dq_acc, void* dq, cudaStream_t st) {
+  const int64_t total = int64_t(p.B) * p.N * p.Sq * p.D;
+  const int g = grid_for(total, 256);
+  if (is_bf16)
+    bwd_post_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
+        p, dq_acc, static_cast<__nv_bfloat16*>(dq));
+  else
+    bwd_post_kernel<float><<<g, 256, 0, st>>>(p, dq_acc, static_cast<float*>(dq));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_map(const Problem& p, uint8_t* tile_map,
+                            cudaStream_t st) {
+  const int64_t nqt = (p.Sq + FA_TILE_M - 1) / FA_TILE_M;
+  const int64_t nkt = (p.Sk + FA_TILE_N - 1) / FA_TILE_N;
+  const int64_t tiles = int64_t(p.B) * p.tm_heads * nqt * nkt;
+  if (tiles == 0) return cudaSuccess;
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+  tile_map_kernel<<<unsigned(tiles), 256, 0, st>>>(p, tile_map);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_modality_mask(int B, int S, const int32_t* ids,
+                                 uint32_t allow_bits, uint8_t* mask,
+                                 cudaStream_t st) {
+  const int64_t total = int64_t(B) * S * S;
+  if (total == 0) return cudaSuccess;
+  modality_mask_kernel<<<grid_for(total, 256), 256, 0, st>>>(B, S, ids,
+                                                              allow_bits, mask);
+  return cudaGetLastError();
+}
+
+}  // namespace fa

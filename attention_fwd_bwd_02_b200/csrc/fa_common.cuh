@@ -1,0 +1,80 @@
+// fa_common.cuh -- problem description shared by the host launcher and all
+// kernels, and the visibility rule of one (query, key) pair.
+#pragma once
+
+#include <stdint.h>
+
+#include "../../include/fa.h"
+
+namespace fa {
+
+// Everything a kernel needs to know about one call.  Strides are in
+// elements; element (b, h, s, d) of q/out/dout sits at
+//   b*q_sb + h*q_sh + s*q_ss + d   (k/v/dk/dv alike with k_*).
+struct Problem {
+  int B, N, Sq, Sk, D;
+  int layout;         // FA_LAYOUT_BNSD or FA_LAYOUT_BSH
+  int64_t q_sb, q_sh, q_ss;
+  int64_t k_sb, k_sh, k_ss;
+  float scale;        // multiplies Q.K
+  float scale_log2;   // scale * log2(e)
+  uint32_t mask_flags;
+  const int32_t* kv_len;
+  const uint8_t* mask;
+  int64_t m_sb, m_sh, m_sq;
+  const uint8_t* tile_map;  // [B][tm_heads][q tiles][k tiles] or null
+  int tm_heads;
+  const int32_t* ids;       // modality ids [B][Sk]
+  uint32_t allow_bits;      // bit (2*id_q + id_k): allowed; bit 4: diagonal
+  const float* slopes;      // ALiBi slopes [N] or null
+  uint32_t debug_flags;     // test hooks (include/fa_testing.h)
+  unsigned int* status;     // device status word (bit 0: a wait timed out)
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Number of keys of batch b that may be visible at all (padding rule).
+__device__ __forceinline__ int visible_keys(const Problem& p, int b) {
+  int n = p.Sk;
+  if (p.mask_flags & FA_MASK_KV_PADDING) {
+    int kl = p.kv_len[b];
+    n = kl < n ? (kl < 0 ? 0 : kl) : n;
+  }
+  return n;
+}
+
+// Modality rule for ids a (query) and c (key) at positions i, j.
+__device__ __forceinline__ bool modality_ok(uint32_t allow_bits, int a, int c,
+                                            int i, int j) {
+  bool ok = (allow_bits >> ((a & 1) * 2 + (c & 1))) & 1u;
+  if ((allow_bits & 16u) && i == j) ok = true;
+  return ok;
+}
+
+// Visibility of key j for query i in (b, h), all rules; nkeys is
+// visible_keys(p, b).
+__device__ __forceinline__ bool pair_visible(const Problem& p, int b, int h,
+                                             int i, int j, int nkeys) {
+  if (j >= nkeys) return false;
+  if ((p.mask_flags & FA_MASK_CAUSAL) && j > i) return false;
+  if (p.mask_flags & FA_MASK_BOOL) {
+    if (p.mask[b * p.m_sb + h * p.m_sh + int64_t(i) * p.m_sq + j] == 0)
+      return false;
+  }
+  if (p.mask_flags & FA_MASK_MODALITY) {
+    const int32_t* id = p.ids + int64_t(b) * p.Sk;
+    if (!modality_ok(p.allow_bits, id[i], id[j], i, j)) return false;
+  }
+  return true;
+}
+
+// ALiBi bias of (h, i, j) in natural units: -slope_h * |i - j|.
+__device__ __forceinline__ float alibi_bias(const Problem& p, int h, int i,
+                                            int j) {
+  int d = i - j;
+  d = d < 0 ? -d : d;
+  return -p.slopes[h] * float(d);
+}
+
+}  // namespace fa

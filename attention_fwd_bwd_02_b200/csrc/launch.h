@@ -1,0 +1,43 @@
+// launch.h -- host-side launchers of the kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "fa_common.cuh"
+
+namespace fa {
+
+// fp32 FMA path (simt.cu).
+cudaError_t launch_fwd_f32(const Problem& p, const void* q, const void* k,
+                           const void* v, void* out, float* lse,
+                           cudaStream_t st);
+cudaError_t launch_bwd_f32(const Problem& p, const void* q, const void* k,
+                           const void* v, const void* dout, const float* lse,
+                           const float* delta, float* dq_acc, void* dk,
+                           void* dv, cudaStream_t st);
+
+// bf16 tensor-core path (fwd_sm100.cu, bwd_sm100.cu).
+cudaError_t launch_fwd_bf16_sm100(const Problem& p, const void* q,
+                                  const void* k, const void* v, void* out,
+                                  float* lse, cudaStream_t st);
+cudaError_t launch_bwd_bf16_sm100(const Problem& p, const void* q,
+                                  const void* k, const void* v,
+                                  const void* dout, const float* lse,
+                                  const float* delta, float* dq_acc, void* dk,
+                                  void* dv, cudaStream_t st);
+
+// Helpers (aux.cu).  is_bf16 selects the element type of the tensors.
+cudaError_t launch_bwd_pre(const Problem& p, bool is_bf16, const void* out,
+                           const void* dout, float* delta, float* dq_acc,
+                           cudaStream_t st);
+cudaError_t launch_bwd_post(const Problem& p, bool is_bf16,
+                            const float* dq_acc, void* dq, cudaStream_t st);
+cudaError_t launch_fill_empty_rows(const Problem& p, bool is_bf16, void* out,
+                                   float* lse, cudaStream_t st);
+cudaError_t launch_tile_map(const Problem& p, uint8_t* tile_map,
+                            cudaStream_t st);
+cudaError_t launch_modality_mask(int B, int S, const int32_t* ids,
+                                 uint32_t allow_bits, uint8_t* mask,
+                                 cudaStream_t st);
+
+}  // namespace fa

@@ -1,0 +1,63 @@
+// tma_host.cu -- cuTensorMapEncodeTiled through the runtime's driver entry
+// point (no link-time dependency on libcuda).
+#include "tma_host.h"
+
+#include <mutex>
+
+namespace fa {
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
+                                   void*, const cuuint64_t*, const cuuint64_t*,
+                                   const cuuint32_t*, const cuuint32_t*,
+                                   CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion,
+                                   CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr,
+                                cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t make_operand_map(CUtensorMap* map, const void* base,
+                             const Problem& p, int S, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return cudaErrorNotSupported;
+  cuuint64_t dims[3], strides[2];
+  const cuuint64_t esz = 2;  // bf16
+  if (p.layout == FA_LAYOUT_BSH) {
+    dims[0] = cuuint64_t(p.N) * p.D;
+    dims[1] = cuuint64_t(S);
+    dims[2] = cuuint64_t(p.B);
+    strides[0] = dims[0] * esz;
+    strides[1] = dims[0] * dims[1] * esz;
+  } else {
+    dims[0] = cuuint64_t(p.D);
+    dims[1] = cuuint64_t(S);
+    dims[2] = cuuint64_t(p.B) * p.N;
+    strides[0] = dims[0] * esz;
+    strides[1] = dims[0] * dims[1] * esz;
+  }
+  const cuuint32_t box[3] = {64u, cuuint32_t(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                   const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace fa

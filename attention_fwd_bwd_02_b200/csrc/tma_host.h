@@ -1,0 +1,20 @@
+// tma_host.h -- host-side construction of TMA tensor maps for the bf16
+// operands (Q, K, V, dO, ...).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "fa_common.cuh"
+
+namespace fa {
+
+// Tensor map over a bf16 operand with S rows per head, read as boxes of
+// 64 columns x box_rows rows with 128-byte swizzle (the canonical K-major /
+// MN-major operand layout of tcgen05).  Coordinates (x, row, z):
+//   BNSD: x = column 0..D-1, z = b*N + h;   BSH: x = h*D + column, z = b.
+// Rows past S read as zeros.
+cudaError_t make_operand_map(CUtensorMap* map, const void* base,
+                             const Problem& p, int S, int box_rows);
+
+}  // namespace fa

@@ -1,0 +1,177 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) fused attention library libfa_b200.so.
+ *
+ * The operation is masked softmax attention with an optional position bias,
+ *
+ *     out = Softmax(Q K^T * scale + atten_mask + pse) V,
+ *
+ * as stated by the FlashAttentionScore fusion-operator guide ("operator
+ * mathematics", sec. 2, and the call npu_fusion_attention(query, key, value,
+ * head_num, input_layout, pse, padding_mask, atten_mask, scale, keep_prob) of
+ * its sec. 3.1 with the parameter table of sec. 3.2).  The N x N score matrix
+ * is never written to memory: it is built tile by tile with an online softmax
+ * (same guide, sec. 2), and the backward pass recomputes the probabilities
+ * from the per-row log-sum-exp saved by the forward.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor pointers are DEVICE pointers, allocated and owned by the
+ *    caller.  The library never allocates device memory and keeps no state
+ *    between calls, except one device-side status word (fa_sync_status).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  Every call that launches work is asynchronous on that stream.
+ *  - Argument errors are detected on the host before anything is launched
+ *    and returned synchronously; nothing is written in that case.
+ *  - A failed launch returns FA_ERR_CUDA.  Errors inside a running kernel
+ *    (a bounded wait that gave up) are recorded in the status word and
+ *    reported by fa_sync_status.
+ *  - Layouts (input_layout of the guide, sec. 3.2):
+ *      FA_LAYOUT_BNSD: q is [B][N][Sq][D], k and v are [B][N][Sk][D].
+ *      FA_LAYOUT_BSH : q is [B][Sq][H], k and v are [B][Sk][H] with
+ *                      H = N * D and head h at columns h*D .. h*D+D-1.
+ *    All contiguous, D innermost.  out, dq, dk, dv use the layout and dtype
+ *    of q, k, v.  lse is always fp32 [B][N][Sq].
+ *  - Dtypes: FA_BF16 (tensor-core path, D in {64, 128}) or FA_F32 (fp32 FMA
+ *    path, 1 <= D <= 128).  Accumulation is fp32 in both.
+ *  - Tensor pointers must be 16-byte aligned.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* malformed argument (null, shape, stride)      */
+  FA_ERR_UNSUPPORTED = 2,  /* well-formed but not implemented (keep_prob<1) */
+  FA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed          */
+  FA_ERR_TIMEOUT = 4       /* a kernel's bounded wait gave up               */
+} fa_status;
+
+typedef enum { FA_LAYOUT_BNSD = 0, FA_LAYOUT_BSH = 1 } fa_layout;
+typedef enum { FA_F32 = 0, FA_BF16 = 1 } fa_dtype;
+
+/* Mask rules (bit flags, combinable).  A key j is visible to query i when
+ * every active rule allows it.  Disallowed scores are -inf before the
+ * softmax (masked_fill with -inf of the multimodal FlashAttention page,
+ * layer 2).  A row with no visible key returns out = 0 and lse = -inf, and
+ * contributes nothing to the gradients. */
+enum {
+  FA_MASK_CAUSAL = 1,      /* j <= i, top-left aligned (the lower-triangular
+                              tril mask of the CogVLM page, "attention mask
+                              mechanism")                                    */
+  FA_MASK_KV_PADDING = 2,  /* j < kv_len[b] (key-side document padding mask,
+                              retrieval page, layer 2 SemanticModeler)       */
+  FA_MASK_BOOL = 4,        /* mask[b,h,i,j] != 0, 1 = may attend (polarity of
+                              create_cross_modal_mask, multimodal page)      */
+  FA_MASK_MODALITY = 8     /* allow[id_i][id_j] || (allow_diag && i == j),
+                              ids = modality_ids[b][*] in {0, 1}; the
+                              cross-modal rule of the multimodal page as a
+                              2x2 table, evaluated on the fly (Sq == Sk)    */
+};
+
+/* Granularity of the optional tile map (rows x keys of one tile). */
+enum { FA_TILE_M = 128, FA_TILE_N = 128 };
+
+typedef struct {
+  uint32_t flags;               /* OR of FA_MASK_*                           */
+  const int32_t* kv_len;        /* [B] device, FA_MASK_KV_PADDING            */
+  const uint8_t* mask;          /* device, FA_MASK_BOOL; element (b,h,i,j) at
+                                   b*stride_b + h*stride_h + i*stride_q + j;
+                                   a zero stride broadcasts that axis        */
+  int64_t mask_stride_b, mask_stride_h, mask_stride_q;
+  const uint8_t* tile_map;      /* optional, from fa_build_mask_tile_map for
+                                   this very mask and shape: lets the kernels
+                                   skip tiles with no visible key.  NULL =
+                                   treat every tile as partially visible.    */
+  const int32_t* modality_ids;  /* [B][S] device, FA_MASK_MODALITY          */
+  uint8_t allow[2][2];          /* allow[id_q][id_k], FA_MASK_MODALITY      */
+  uint8_t allow_diag;           /* also allow i == j, FA_MASK_MODALITY      */
+} fa_mask;
+
+/* Position bias `pse` (guide, sec. 3.2: "optional, supports fusing position
+ * encodings such as ALiBi").  FA_PSE_ALIBI adds -slopes[h] * |i - j| to the
+ * scaled score; the bias is not multiplied by `scale`. */
+enum { FA_PSE_NONE = 0, FA_PSE_ALIBI = 1 };
+typedef struct {
+  int kind;                     /* FA_PSE_*                                  */
+  const float* slopes;          /* [N] device, FA_PSE_ALIBI                  */
+} fa_pse;
+
+typedef struct {
+  int B, N, Sq, Sk, D;          /* batch, heads (head_num), query and key
+                                   lengths, head dim                         */
+  fa_layout layout;
+  fa_dtype dtype;
+} fa_shape;
+
+/* Forward.  Writes out (layout/dtype of q) and lse (fp32 [B][N][Sq], natural
+ * log, -inf for rows with no visible key).
+ *   pse, mask : may be NULL (no bias / no mask).
+ *   scale     : multiplies Q K^T (the 1/sqrt(d_k) of the guide's table; no
+ *               default is assumed).
+ *   keep_prob : must be 1.0 (no dropout); anything else returns
+ *               FA_ERR_UNSUPPORTED.
+ * Errors: FA_ERR_INVALID_ARG for null tensors, non-positive sizes, a
+ * modality mask with Sq != Sk or a missing mask pointer; FA_ERR_UNSUPPORTED
+ * for keep_prob != 1 or a bf16 head dim other than 64 / 128. */
+fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
+                 const void* v, const fa_pse* pse, const fa_mask* mask,
+                 float scale, float keep_prob, void* out, float* lse,
+                 void* stream);
+
+/* Bytes of device workspace fa_bwd needs for this shape (fp32 dQ
+ * accumulator plus per-row fp32 statistics).  0 on invalid shapes. */
+size_t fa_bwd_workspace_size(const fa_shape* shape);
+
+/* Backward: gradients of sum(dout * out) with respect to q, k and v, given
+ * the forward's out and lse.  workspace must hold fa_bwd_workspace_size()
+ * bytes (16-byte aligned); its contents on entry do not matter.  dq, dk, dv
+ * are fully overwritten.  No gradient is produced for pse or the mask.
+ * Errors as fa_fwd, plus FA_ERR_INVALID_ARG for a short workspace. */
+fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
+                 const void* v, const void* out, const void* dout,
+                 const float* lse, const fa_pse* pse, const fa_mask* mask,
+                 float scale, float keep_prob, void* dq, void* dk, void* dv,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of the tile map for FA_MASK_BOOL with this shape and mask strides:
+ * one byte per (b, h or 1 when mask_stride_h == 0, query tile, key tile). */
+size_t fa_mask_tile_map_size(const fa_shape* shape, const fa_mask* mask);
+
+/* Classifies every FA_TILE_M x FA_TILE_N tile of the bool mask as
+ * 0 = no visible key, 1 = partly visible, 2 = fully visible, into
+ * tile_map (fa_mask_tile_map_size bytes, device).  Reads the mask once. */
+fa_status fa_build_mask_tile_map(const fa_shape* shape, const fa_mask* mask,
+                                 uint8_t* tile_map, void* stream);
+
+/* Builds the explicit cross-modal bool mask [B][S][S] (u8, 1 = may attend)
+ * from modality_ids [B][S] with the 2x2 allow table and diagonal rule of
+ * FA_MASK_MODALITY (the multimodal page's create_cross_modal_mask,
+ * generalised).  Use with mask_stride_b = S*S, mask_stride_h = 0,
+ * mask_stride_q = S. */
+fa_status fa_build_modality_mask(int B, int S, const int32_t* modality_ids,
+                                 const uint8_t allow[2][2], int allow_diag,
+                                 uint8_t* mask_out, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device status word:
+ * FA_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call,
+ * FA_ERR_CUDA if the stream reported an error, else FA_OK. */
+fa_status fa_sync_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* fa_status_string(fa_status status);
+
+/* Library version string, e.g. "fa_b200 1.0 sm_100a". */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */
