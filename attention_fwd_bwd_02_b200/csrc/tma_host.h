@@ -17,4 +17,11 @@ namespace fa {
 cudaError_t make_operand_map(CUtensorMap* map, const void* base,
                              const Problem& p, int S, int box_rows);
 
+// Tensor map over an fp32 [planes][rows][cols] array (cols contiguous),
+// boxes of box_cols x box_rows, no swizzle.  Used for the tiled reduce-add
+// into the dQ accumulator; elements outside the array are skipped.
+cudaError_t make_f32_rows_map(CUtensorMap* map, const void* base, int cols,
+                              int rows, int64_t planes, int box_cols,
+                              int box_rows);
+
 }  // namespace fa
