@@ -130,6 +130,15 @@ unsigned int* status_word() {
   return addr[dev];
 }
 
+// Last CUDA error seen by an entry point of this thread (diagnostics only).
+thread_local cudaError_t g_last_cuda = cudaSuccess;
+
+fa_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return FA_OK;
+  g_last_cuda = e;
+  return FA_ERR_CUDA;
+}
+
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 size_t elem_size(const fa_shape* s) { return s->dtype == FA_BF16 ? 2 : 4; }
@@ -151,6 +160,8 @@ const char* fa_status_string(fa_status status) {
 
 const char* fa_version(void) { return "fa_b200 1.0 sm_100a"; }
 
+const char* fa_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
+
 fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
                  const void* v, const fa_pse* pse, const fa_mask* mask,
                  float scale, float keep_prob, void* out, float* lse,
@@ -160,7 +171,7 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
   if (st != FA_OK) return st;
   if (p.B == 0 || p.N == 0 || p.Sq == 0) return FA_OK;  // nothing to write
   p.status = status_word();
-  if (!p.status) return FA_ERR_CUDA;
+  if (!p.status) return cuda_status(cudaErrorNoDevice);
   if (!q || !out || !lse || (p.Sk > 0 && (!k || !v))) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(out) || (p.Sk > 0 && (!aligned16(k) || !aligned16(v))) ||
       (reinterpret_cast<uintptr_t>(lse) & 3u))
@@ -174,7 +185,7 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
     e = fa::launch_fwd_bf16_sm100(p, q, k, v, out, lse, cs);
   else
     e = fa::launch_fwd_f32(p, q, k, v, out, lse, cs);
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 size_t fa_bwd_workspace_size(const fa_shape* shape) {
@@ -200,14 +211,15 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
     if (p.Sq == 0 && p.Sk > 0) {
       if (!dk || !dv) return FA_ERR_INVALID_ARG;
       const size_t n = size_t(p.B) * p.N * p.Sk * p.D * es;
-      if (cudaMemsetAsync(dk, 0, n, cs) != cudaSuccess ||
-          cudaMemsetAsync(dv, 0, n, cs) != cudaSuccess)
-        return FA_ERR_CUDA;
+      cudaError_t e = cudaMemsetAsync(dk, 0, n, cs);
+      if (e == cudaSuccess) e = cudaMemsetAsync(dv, 0, n, cs);
+      if (e != cudaSuccess) return cuda_status(e);
     }
     if (p.Sk == 0 && p.Sq > 0) {
       if (!dq) return FA_ERR_INVALID_ARG;
       const size_t n = size_t(p.B) * p.N * p.Sq * p.D * es;
-      if (cudaMemsetAsync(dq, 0, n, cs) != cudaSuccess) return FA_ERR_CUDA;
+      cudaError_t e = cudaMemsetAsync(dq, 0, n, cs);
+      if (e != cudaSuccess) return cuda_status(e);
     }
     return FA_OK;
   }
@@ -219,7 +231,7 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
     return FA_ERR_INVALID_ARG;
   if (workspace_bytes < fa_bwd_workspace_size(shape)) return FA_ERR_INVALID_ARG;
   p.status = status_word();
-  if (!p.status) return FA_ERR_CUDA;
+  if (!p.status) return cuda_status(cudaErrorNoDevice);
   const size_t rows = size_t(p.B) * p.N * p.Sq;
   float* dq_acc = static_cast<float*>(workspace);
   float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
@@ -233,7 +245,7 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
       e = fa::launch_bwd_f32(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, cs);
   }
   if (e == cudaSuccess) e = fa::launch_bwd_post(p, bf16, dq_acc, dq, cs);
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 size_t fa_mask_tile_map_size(const fa_shape* shape, const fa_mask* mask) {
@@ -252,7 +264,7 @@ fa_status fa_build_mask_tile_map(const fa_shape* shape, const fa_mask* mask,
   if (st != FA_OK) return st;
   if (!mask || !(mask->flags & FA_MASK_BOOL) || !tile_map) return FA_ERR_INVALID_ARG;
   cudaError_t e = fa::launch_tile_map(p, tile_map, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 fa_status fa_build_modality_mask(int B, int S, const int32_t* modality_ids,
@@ -266,18 +278,20 @@ fa_status fa_build_modality_mask(int B, int S, const int32_t* modality_ids,
                         (allow_diag ? 16u : 0u);
   cudaError_t e = fa::launch_modality_mask(B, S, modality_ids, bits, mask_out,
                                            static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return cuda_status(e);
 }
 
 fa_status fa_sync_status(void* stream) {
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (cudaStreamSynchronize(cs) != cudaSuccess) return FA_ERR_CUDA;
+  cudaError_t e = cudaStreamSynchronize(cs);
+  if (e != cudaSuccess) return cuda_status(e);
   unsigned int word = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&word, fa::g_fa_status, sizeof(word)) != cudaSuccess)
-    return FA_ERR_CUDA;
-  if (word != 0 &&
-      cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(zero)) != cudaSuccess)
-    return FA_ERR_CUDA;
+  e = cudaMemcpyFromSymbol(&word, fa::g_fa_status, sizeof(word));
+  if (e != cudaSuccess) return cuda_status(e);
+  if (word != 0) {
+    e = cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_status(e);
+  }
   return word ? FA_ERR_TIMEOUT : FA_OK;
 }
 

@@ -27,8 +27,31 @@ __device__ __forceinline__ void from_f(float v, __nv_bfloat16* dst) {
   *dst = __float2bfloat16_rn(v);
 }
 
-// One warp per query row: Delta = dot(dO_i, O_i).  Also clears the row of the
-// dQ accumulator ([B][N][Sq][D] fp32).
+// Four consecutive elements (D % 4 == 0 keeps them inside one row and
+// 8/16-byte aligned).
+__device__ __forceinline__ float4 load4(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
+  return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+}
+__device__ __forceinline__ void store4(float* p, float4 v) {
+  *reinterpret_cast<float4*>(p) = v;
+}
+__device__ __forceinline__ void store4(__nv_bfloat16* p, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+  __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
+}
+
+// One warp per query row (grid-strided): Delta = dot(dO_i, O_i), and the
+// row of the fp32 dQ accumulator ([B][N][Sq][D]) is cleared.
 template <typename T>
 __global__ void bwd_pre_kernel(Problem p, const T* __restrict__ out,
                                const T* __restrict__ dout,
@@ -37,6 +60,7 @@ __global__ void bwd_pre_kernel(Problem p, const T* __restrict__ out,
   const int lane = threadIdx.x & 31;
   const int64_t rows = int64_t(p.B) * p.N * p.Sq;
   const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  const bool vec = (p.D & 3) == 0;
   for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
        r < rows; r += warps) {
     const int i = int(r % p.Sq);
@@ -44,29 +68,49 @@ __global__ void bwd_pre_kernel(Problem p, const T* __restrict__ out,
     const int h = int(bh % p.N), b = int(bh / p.N);
     const int64_t off = b * p.q_sb + h * p.q_sh + int64_t(i) * p.q_ss;
     float acc = 0.f;
-    for (int d = lane; d < p.D; d += 32)
-      acc = fmaf(to_f(dout[off + d]), to_f(out[off + d]), acc);
+    float* z = dq_acc + r * p.D;
+    if (vec) {
+      for (int d = lane * 4; d < p.D; d += 128) {
+        const float4 a = load4(dout + off + d), o = load4(out + off + d);
+        acc += a.x * o.x + a.y * o.y + a.z * o.z + a.w * o.w;
+        store4(z + d, make_float4(0.f, 0.f, 0.f, 0.f));
+      }
+    } else {
+      for (int d = lane; d < p.D; d += 32) {
+        acc = fmaf(to_f(dout[off + d]), to_f(out[off + d]), acc);
+        z[d] = 0.f;
+      }
+    }
 #pragma unroll
     for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(~0u, acc, o);
     if (lane == 0) delta[r] = acc;
-    float* z = dq_acc + r * p.D;
-    for (int d = lane; d < p.D; d += 32) z[d] = 0.f;
   }
 }
 
+// One warp per query row: dQ = scale * dQacc in the tensor dtype / layout.
 template <typename T>
 __global__ void bwd_post_kernel(Problem p, const float* __restrict__ dq_acc,
                                 T* __restrict__ dq) {
-  const int64_t total = int64_t(p.B) * p.N * p.Sq * p.D;
-  for (int64_t e = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; e < total;
-       e += int64_t(gridDim.x) * blockDim.x) {
-    const int d = int(e % p.D);
-    const int64_t r = e / p.D;
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  const int64_t warps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  const bool vec = (p.D & 3) == 0;
+  for (int64_t r = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+       r < rows; r += warps) {
     const int i = int(r % p.Sq);
     const int64_t bh = r / p.Sq;
     const int h = int(bh % p.N), b = int(bh / p.N);
-    from_f(dq_acc[e] * p.scale,
-           dq + b * p.q_sb + h * p.q_sh + int64_t(i) * p.q_ss + d);
+    T* dst = dq + b * p.q_sb + h * p.q_sh + int64_t(i) * p.q_ss;
+    const float* src = dq_acc + r * p.D;
+    if (vec) {
+      for (int d = lane * 4; d < p.D; d += 128) {
+        float4 v = load4(src + d);
+        v.x *= p.scale; v.y *= p.scale; v.z *= p.scale; v.w *= p.scale;
+        store4(dst + d, v);
+      }
+    } else {
+      for (int d = lane; d < p.D; d += 32) from_f(src[d] * p.scale, dst + d);
+    }
   }
 }
 
@@ -163,8 +207,8 @@ cudaError_t launch_bwd_pre(const Problem& p, bool is_bf16, const void* out,
 
 cudaError_t launch_bwd_post(const Problem& p, bool is_bf16,
                             const float* dq_acc, void* dq, cudaStream_t st) {
-  const int64_t total = int64_t(p.B) * p.N * p.Sq * p.D;
-  const int g = grid_for(total, 256);
+  const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  const int g = grid_for(rows, 8);
   if (is_bf16)
     bwd_post_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
         p, dq_acc, static_cast<__nv_bfloat16*>(dq));

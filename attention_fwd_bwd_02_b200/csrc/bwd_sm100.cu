@@ -67,8 +67,8 @@ struct BwdCfg {
   // dq_free, acc_done, drain
   static constexpr int kNumBars = 1 + 2 * kStages + 7;
   static constexpr int kSmemMisc = kSmemBar + kNumBars * 8;
-  static constexpr int kSmemQtIds = kSmemMisc + 16;
-  static constexpr int kSmemBytes = kSmemQtIds + kMaxQTiles + 1024;
+  static constexpr int kSmemQtBits = kSmemMisc + 16;  // [qt][2] id==1 bits of queries
+  static constexpr int kSmemBytes = kSmemQtBits + kMaxQTiles * 8 + 1024;
 };
 
 struct KeyCtx {
@@ -80,7 +80,7 @@ struct KeyCtx {
 
 // 0 = no visible pair, 1 = some pairs (mask per element), 2 = all pairs.
 __device__ __forceinline__ int qtile_class(const Problem& p, const KeyCtx& c,
-                                           int qt, const uint8_t* qt_ids) {
+                                           int qt, const uint32_t* qt_bits) {
   const int q0 = qt * kBM;
   const int q_last = min(q0 + kBM, p.Sq) - 1;
   if (c.k0 >= c.nkeys) return 0;
@@ -103,7 +103,15 @@ __device__ __forceinline__ int qtile_class(const Problem& p, const KeyCtx& c,
     }
   }
   if (p.mask_flags & FA_MASK_MODALITY) {
-    const uint32_t qs = qt_ids[qt];
+    // id set of the query tile from its id==1 bits and its valid rows
+    const int nvalid = min(kBM, p.Sq - q0);
+    uint32_t any1 = 0, any0 = 0;
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+      any1 |= qt_bits[qt * 2 + w];
+      any0 |= range_bits(0, nvalid - 1, w) & ~qt_bits[qt * 2 + w];
+    }
+    const uint32_t qs = (any0 ? 1u : 0u) | (any1 ? 2u : 0u);
     bool any = false, all = true;
 #pragma unroll
     for (int a = 0; a < 2; ++a)
@@ -158,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kSmemMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kSmemMisc + 4);
-  uint8_t* qt_ids = smem + C::kSmemQtIds;
+  uint32_t* qt_bits = reinterpret_cast<uint32_t*>(smem + C::kSmemQtBits);
 
   const int warp = threadIdx.x >> 5;
   const int tid = threadIdx.x;
@@ -192,11 +200,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (p.mask_flags & FA_MASK_MODALITY) {
     const int32_t* ids = p.ids + int64_t(c.b) * p.Sk;
-    for (int qt = c.qt_begin + tid; qt < c.qt_end; qt += kThreads) {
-      uint32_t set = 0;
-      const int i1 = min(qt * kBM + kBM, p.Sq);
-      for (int i = qt * kBM; i < i1; ++i) set |= 1u << (ids[i] & 1);
-      qt_ids[qt] = uint8_t(set);
+    for (int wq = c.qt_begin * 2 + warp; wq < c.qt_end * 2; wq += kThreads / 32) {
+      const int i = wq * 32 + lane;  // = qt * 64 + w * 32 + lane
+      const bool in = i < p.Sq;
+      const uint32_t is1 = __ballot_sync(~0u, in && (ids[in ? i : 0] & 1) == 1);
+      if (lane == 0) qt_bits[wq] = is1;
     }
     uint32_t ks = 0;
     for (int j = c.k0 + tid; j <= c.k_last; j += kThreads) ks |= 1u << (ids[j] & 1);
@@ -228,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int n = 0;
       for (int qt = c.qt_begin; qt < c.qt_end; ++qt) {
-        if (qtile_class(p, c, qt, qt_ids) == 0) continue;
+        if (qtile_class(p, c, qt, qt_bits) == 0) continue;
         const int st = n % C::kStages, use = n / C::kStages;
         if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&q_full[st], 2 * C::kQTile);
@@ -259,7 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = mbar_wait(kv_full, 0, abort_flag);
       int n = 0;
       for (int qt = c.qt_begin; ok && qt < c.qt_end; ++qt) {
-        if (qtile_class(p, c, qt, qt_ids) == 0) continue;
+        if (qtile_class(p, c, qt, qt_bits) == 0) continue;
         const int st = n % C::kStages;
         if (!mbar_wait(&q_full[st], (n / C::kStages) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -317,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* stage0 = sStage + wq * 2 * (C::kStageBytes / 4);
     int n = 0;
     for (int qt = c.qt_begin; qt < c.qt_end; ++qt) {
-      if (qtile_class(p, c, qt, qt_ids) == 0) continue;
+      if (qtile_class(p, c, qt, qt_bits) == 0) continue;
       const bool got = mbar_wait(dq_full, n & 1, abort_flag);
       if (!__all_sync(~0u, got)) break;
       tc_fence_after();
@@ -364,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int n = 0;
     bool ok = true;
     for (int qt = c.qt_begin; qt < c.qt_end; ++qt) {
-      const int cls = qtile_class(p, c, qt, qt_ids);
+      const int cls = qtile_class(p, c, qt, qt_bits);
       if (cls == 0) continue;
       const int q0 = qt * kBM;
       // Per-row statistics of this query tile (LSE in log2 units), loaded by
@@ -391,6 +399,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait(sr[1]);
       tmem_ld_wait(dr[0]);
       tmem_ld_wait(dr[1]);
+      // Visibility of the 64 queries of this tile for key j, as bits.
+      uint32_t vb[2] = {~0u, ~0u};
+      if (cls == 1) {
+        const int lo = (p.mask_flags & FA_MASK_CAUSAL) ? max(0, j - q0) : 0;
+        const int hi = (j < c.nkeys) ? min(kBM, p.Sq - q0) - 1 : -1;
+        vb[0] = range_bits(lo, hi, 0);
+        vb[1] = range_bits(lo, hi, 1);
+        if (mcol) {
+#pragma unroll 1
+          for (int w = 0; w < 2; ++w) {
+            uint32_t m = 0;
+            for (int e = 0; e < 32 && q0 + 32 * w + e < p.Sq; ++e)
+              m |= uint32_t(mcol[int64_t(q0 + 32 * w + e) * p.m_sq] != 0) << e;
+            vb[w] &= m;
+          }
+        }
+        if (ids) {
+#pragma unroll
+          for (int w = 0; w < 2; ++w) {
+            uint32_t m = modality_row_bits(p.allow_bits, id_j, qt_bits[qt * 2 + w], false);
+            if (p.allow_bits & 16u) m |= range_bits(j - q0, j - q0, w);
+            vb[w] &= m;
+          }
+        }
+      }
       uint32_t pk[32], dk_[32];
 #pragma unroll
       for (int e = 0; e < kBM; e += 2) {
@@ -401,13 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int i = q0 + cc;
           float t = __uint_as_float(sr[cc >> 5][cc & 31]) * sl2;
           if (has_alibi) t = fmaf(-slope_l2, float(abs(i - j)), t);
-          bool vis = true;
-          if (cls == 1) {
-            vis = j < c.nkeys && i < p.Sq;
-            if ((p.mask_flags & FA_MASK_CAUSAL) && j > i) vis = false;
-            if (vis && mcol) vis = mcol[int64_t(i) * p.m_sq] != 0;
-            if (vis && ids) vis = modality_ok(p.allow_bits, ids[i], id_j, i, j);
-          }
+          const bool vis = (vb[cc >> 5] >> (cc & 31)) & 1u;
           const float pp = vis ? ex2_approx(t - st_lse[cc]) : 0.f;
           pv[u] = pp;
           dsv[u] = pp * (__uint_as_float(dr[cc >> 5][cc & 31]) - st_dl[cc]);

@@ -69,6 +69,28 @@ __device__ __forceinline__ bool pair_visible(const Problem& p, int b, int h,
   return true;
 }
 
+// Bits [lo, hi] (inclusive, positions counted from 0) that fall in 32-bit
+// word w of a bit row, i.e. positions 32w .. 32w+31.
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi, int w) {
+  const int a = max(lo - 32 * w, 0), b = min(hi - 32 * w, 31);
+  if (a > b) return 0u;
+  const uint32_t upto_b = (b == 31) ? ~0u : ((2u << b) - 1u);
+  return upto_b & ~((1u << a) - 1u);
+}
+
+// Modality rule as bits: `is1` has bit e set when the id at position e is 1;
+// the row's own id selects which ids it may attend.
+__device__ __forceinline__ uint32_t modality_row_bits(uint32_t allow_bits,
+                                                      int id_row, uint32_t is1,
+                                                      bool row_is_query) {
+  // allow[id_q][id_k]: for a query row, vary id_k; for a key row, vary id_q.
+  const bool to1 = row_is_query ? ((allow_bits >> ((id_row & 1) * 2 + 1)) & 1u)
+                                : ((allow_bits >> (2 + (id_row & 1))) & 1u);
+  const bool to0 = row_is_query ? ((allow_bits >> ((id_row & 1) * 2)) & 1u)
+                                : ((allow_bits >> (id_row & 1)) & 1u);
+  return (to1 ? is1 : 0u) | (to0 ? ~is1 : 0u);
+}
+
 // ALiBi bias of (h, i, j) in natural units: -slope_h * |i - j|.
 __device__ __forceinline__ float alibi_bias(const Problem& p, int h, int i,
                                             int j) {

@@ -97,6 +97,7 @@ def lib():
         L.fa_status_string.argtypes = [ctypes.c_int]
         L.fa_status_string.restype = ctypes.c_char_p
         L.fa_version.restype = ctypes.c_char_p
+        L.fa_last_cuda_error.restype = ctypes.c_char_p
         for fn in (L.fa_fwd, L.fa_bwd, L.fa_build_mask_tile_map,
                    L.fa_build_modality_mask, L.fa_sync_status):
             fn.restype = ctypes.c_int
@@ -113,6 +114,8 @@ def declared_functions(header: str = HEADER):
 
 def _check(status, what):
     if status != FA_OK:
+        if status == FA_ERR_CUDA:
+            what = f"{what} [{lib().fa_last_cuda_error().decode()}]"
         raise FaError(status, what)
 
 

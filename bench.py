@@ -1,0 +1,429 @@
+"""Benchmark of the fused attention hot path (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one forward and one backward pass (every stage of the hot path)
+over one batch of the causal decoder workload: BNSD bf16, B=4, N=32,
+S=2048, D=128, scale 1/sqrt(128), causal mask, dO ~ N(0, 1).  Inputs are
+synthetic, seeded, and resident in HBM; together they exceed the 126 MB L2,
+so no flush is needed between steps.
+
+FLOPs follow the usual convention: 4*B*N*Sq*Sk*D for the forward, 2.5x that
+for the backward, halved under the causal mask.  The metric is whole-job
+TFLOP/s (fwd+bwd), with the forward-only rate and both fractions of the
+measured dense bf16 tensor peak reported alongside.
+
+--impl reference times the fp64 CPU oracle (the reference implementation of
+the method) on a bounded sample of the same workload on this host's cores.
+
+Multi-GPU (torchrun): every rank runs the same workload on its own GPU (the
+operator shards over (b, h) with no data exchange: replicas, weak scaling);
+timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+B, N, S, D = 4, 32, 2048, 128
+WORKLOAD = "causal self-attention fwd+bwd, BNSD bf16, B=4 N=32 S=2048 D=128"
+METRIC = "fused attention TFLOP/s (fwd, fwd+bwd) and % of B200 dense BF16 peak"
+FWD_FLOPS = 4.0 * B * N * S * S * D / 2.0
+BWD_FLOPS = 2.5 * FWD_FLOPS
+STEP_FLOPS = FWD_FLOPS + BWD_FLOPS
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
+                  "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["attention_fwd_bwd_02_b200/csrc/fwd_sm100.cu",
+                  "attention_fwd_bwd_02_b200/csrc/bwd_sm100.cu",
+                  "attention_fwd_bwd_02_b200/csrc/aux.cu",
+                  "attention_fwd_bwd_02_b200/csrc/ptx.cuh"]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic():
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return {}
+    if d.get("source_hash") != source_hash():
+        return {}
+    return d.get("kernels", {})
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons while timing."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        import torch
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_ours(args):
+    import torch
+    from attention_fwd_bwd_02_b200 import fa
+    from attention_fwd_bwd_02_b200 import inputs as I
+
+    rank, world, local = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    case = I.config2()
+    q, k, v, do = (t.to(dev) for t in (case.q, case.k, case.v, case.dout))
+    scale = case.scale
+    shape = fa.make_shape(q, k, N, "BNSD")
+    ws = torch.empty(fa.bwd_workspace_size(shape), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(B, N, S, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    stream = torch.cuda.current_stream(dev)
+
+    def fwd():
+        fa.fwd(q, k, v, N, "BNSD", scale=scale, causal=True, out=out, lse=lse)
+
+    def bwd():
+        fa.bwd(q, k, v, out, do, lse, N, "BNSD", scale=scale, causal=True,
+               workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    # Clocks are sampled from the warm-up on, so that even a short timed
+    # region sees several samples of the loaded GPU.
+    clk = ClockSampler(local).__enter__()
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    fa.sync_status(dev)
+
+    # --- device-resident timing: per-step events around fwd and bwd
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    if True:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            fwd()
+            ev[s][1].record(stream)
+            bwd()
+            ev[s][2].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    clk.__exit__(None, None, None)
+    fa.sync_status(dev)
+    total_ms = t0.elapsed_time(t1)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+    total_ms = max_over_ranks(total_ms, world)
+    fwd_ms = max_over_ranks(fwd_ms, world)
+    bwd_ms = max_over_ranks(bwd_ms, world)
+    barrier(world)
+
+    # --- end to end through the public API with host buffers
+    pin = {n: t.pin_memory() for n, t in (("q", case.q), ("k", case.k), ("v", case.v),
+                                          ("do", case.dout))}
+    host_out = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                for n, t in (("out", out), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+
+    def e2e_step():
+        q.copy_(pin["q"], non_blocking=True)
+        k.copy_(pin["k"], non_blocking=True)
+        v.copy_(pin["v"], non_blocking=True)
+        do.copy_(pin["do"], non_blocking=True)
+        fwd()
+        bwd()
+        host_out["out"].copy_(out, non_blocking=True)
+        host_out["lse"].copy_(lse, non_blocking=True)
+        host_out["dq"].copy_(dq, non_blocking=True)
+        host_out["dk"].copy_(dk, non_blocking=True)
+        host_out["dv"].copy_(dv, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    fa.sync_status(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / args.steps
+
+    if rank != 0:
+        finish(world)
+        return
+    pk, pk_kind = peaks()
+    ms_step = total_ms / args.steps
+    value = STEP_FLOPS * world / (ms_step * 1e-3) / 1e12
+    fwd_tf = FWD_FLOPS / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = BWD_FLOPS / (bwd_ms * 1e-3) / 1e12
+    peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    peak_sust = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    traffic = committed_traffic()
+    dominant = "bwd" if bwd_ms >= fwd_ms else "fwd"
+
+    def roof(kind, tf, ms):
+        return {"kernel": "fa_fwd (fwd_bf16_sm100)" if kind == "fwd" else
+                "fa_bwd (bwd_pre + bwd_bf16_sm100 + bwd_post)",
+                "bound": "tensor", "achieved": round(tf, 1), "peak": peak_burst,
+                "unit": "TFLOP/s", "frac": round(tf / peak_burst, 4),
+                "peak_kind": f"{pk_kind} bf16_tflops (burst)",
+                "frac_of_sustained": round(tf / peak_sust, 4),
+                "frac_of_nominal_2250": round(tf / 2250.0, 4),
+                "ms_per_launch": round(ms, 4),
+                "algorithmic_flops": FWD_FLOPS if kind == "fwd" else BWD_FLOPS,
+                "traffic": traffic.get(kind)}
+
+    cpu = cpu_baseline(args) if not args.no_cpu_baseline else None
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1), resident in HBM)",
+        "config": {"workload": WORKLOAD, "B": B, "N": N, "S": S, "D": D,
+                   "mask": "causal", "scale": "1/sqrt(128)",
+                   "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": "inputs exceed L2 (335 MB > 126 MB), no flush"},
+        "fwd_tflops": round(fwd_tf, 2),
+        "bwd_tflops": round(bwd_tf, 2),
+        "fwd_ms": round(fwd_ms, 4),
+        "bwd_ms": round(bwd_ms, 4),
+        "fwd_frac_of_peak": round(fwd_tf / peak_burst, 4),
+        "fwd_frac_of_nominal_2250": round(fwd_tf / 2250.0, 4),
+        "roofline": roof(dominant, bwd_tf if dominant == "bwd" else fwd_tf,
+                         bwd_ms if dominant == "bwd" else fwd_ms),
+        "roofline_fwd": roof("fwd", fwd_tf, fwd_ms),
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(STEP_FLOPS * world / (e2e_ms * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(e2e_ms, 4)},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    finish(world)
+
+
+def finish(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def oracle_sample(n_heads, seq):
+    """fwd+bwd of the oracle on n_heads heads of the workload's operator
+    (causal, D=128, scale 1/sqrt(128)) over a seq-token prefix.  Returns
+    (seconds, algorithmic flops of the sample, threads used)."""
+    import oracle
+    from attention_fwd_bwd_02_b200 import inputs as I
+    case = I.make_case("oracle_sample", 1, n_heads, seq, seq, D, seed=1002, causal=True)
+    f64 = lambda t: t.double().numpy()
+    q, k, v, do = f64(case.q), f64(case.k), f64(case.v), f64(case.dout)
+    threads = min(len(os.sched_getaffinity(0)), n_heads)
+    oracle.set_threads(threads)
+    t = time.perf_counter()
+    oracle.fwd(q, k, v, case.scale, causal=True)
+    oracle.bwd(q, k, v, do, case.scale, causal=True)
+    dt = time.perf_counter() - t
+    flops = 3.5 * 4.0 * n_heads * seq * seq * D / 2.0
+    return dt, flops, threads
+
+
+def sample_heads(args, per_core):
+    if args.cpu_heads > 0:
+        return args.cpu_heads
+    return per_core * len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(args):
+    n = sample_heads(args, 24)
+    dt, flops, threads = oracle_sample(n, args.cpu_seq)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{n} heads of the workload's operator (causal, D={D}) over a "
+                      f"{args.cpu_seq}-token prefix, fwd+bwd in fp64, {dt:.1f} s",
+            "seconds": round(dt, 2)}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    times, flops_s = [], 0.0
+    n = sample_heads(args, 1)
+    threads = 1
+    for _ in range(min(args.warmup, 1)):
+        oracle_sample(1, args.cpu_seq)
+    for _ in range(args.steps):
+        dt, fl, threads = oracle_sample(n, args.cpu_seq)
+        times.append(dt)
+        flops_s = fl
+    ms = 1e3 * sum(times) / len(times)
+    value = flops_s / (ms * 1e-3) / 1e12
+    line = {
+        "impl": "reference",
+        "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic (seeded N(0,1))",
+        "config": {"workload": WORKLOAD, "B": B, "N": N, "S": S, "D": D,
+                   "mask": "causal", "parallelism": "host cores (OpenMP over heads)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                         "kind": "oracle",
+                         "sample": f"each step: {n} heads of the workload's operator "
+                                   f"(causal, D={D}) over a {args.cpu_seq}-token prefix, "
+                                   "fwd+bwd in fp64"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-heads", type=int, default=0,
+                    help="(b, h) heads in the oracle's bounded sample "
+                         "(default: one per host core)")
+    ap.add_argument("--cpu-seq", type=int, default=512,
+                    help="token prefix of the oracle's bounded sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "ours":
+        args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -170,6 +170,10 @@ const char* fa_status_string(fa_status status);
 /* Library version string, e.g. "fa_b200 1.0 sm_100a". */
 const char* fa_version(void);
 
+/* Text of the last CUDA error behind an FA_ERR_CUDA returned to the calling
+ * thread ("no error" if none).  Static storage; diagnostics only. */
+const char* fa_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif
