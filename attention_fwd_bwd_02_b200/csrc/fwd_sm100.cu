@@ -5,19 +5,23 @@
 // sec. 2 formula; sec. 3.2 parameters), tile by tile with an online softmax
 // so the score matrix never leaves the SM.
 //
-// One CTA owns two 128-row query tiles (256 rows) of one (b, h) and walks the
-// key tiles (128 keys each) that its mask leaves visible.  The two query
+// Persistent kernel: one CTA per SM walks a static list of work items.  A
+// work item is two 128-row query tiles (256 rows) of one (b, h); the CTA walks
+// the key tiles (128 keys each) that the mask leaves visible.  The two query
 // tiles ping-pong on the tensor core: while the softmax warps of one tile
-// turn S into P, the tensor core runs P V and Q K^T of the other.
+// turn S into P, the tensor core runs P V and Q K^T of the other.  Items are
+// ordered longest first under the causal mask and dealt round-robin, so the
+// CTAs finish together; the loads of the next item overlap the tail of the
+// current one.
 // Warp roles:
 //   warps 0-3 / 4-7  softmax of query tile 0 / 1: thread t owns query row t.
 //              Reads S from TMEM, applies scale / ALiBi / mask, updates the
 //              running max and sum, writes P (bf16) back into TMEM over S,
 //              rescales O in TMEM when the running max grew by more than
-//              2^8, and finally writes O / l and the LSE.
-//   warp 8     TMA producer: both Q tiles once, then K_j and V_j through two
-//              separate rings of stages.
-//   warp 9     MMA issuer (one elected thread) and TMEM owner:
+//              2^8, and at the end of an item writes O / l and the LSE.
+//   warp 8     TMA producer: both Q tiles per item, then K_j and V_j through
+//              two separate rings of stages.
+//   warp 9     MMA issuer (one elected lane) and TMEM owner:
 //              S_t = Q_t K_j^T (SS form), O_t += P_t V_j (P from TMEM, TS form).
 //   warps 10-11 idle (they complete the third warpgroup, which gives its
 //              registers to the softmax warpgroups).
@@ -42,11 +46,16 @@ namespace fa {
 namespace {
 
 constexpr int kBM = 128;              // query rows per tile
-constexpr int kTiles = 2;             // query tiles per CTA
-constexpr int kRows = kBM * kTiles;   // query rows per CTA
+constexpr int kTiles = 2;             // query tiles per work item
+constexpr int kRows = kBM * kTiles;   // query rows per work item
 constexpr int kBN = 128;              // keys per tile
 constexpr int kBoxBytes = 128 * 128;  // one 128-row x 64-col bf16 box
-constexpr int kThreads = 384;  // 3 warpgroups
+constexpr int kThreads = 384;         // 3 warpgroups
+constexpr int kTmemCols = 512;
+constexpr float kRescaleLog2 = 8.0f;  // rescale O only if max grows > 2^8
+constexpr int kSchedRing = 4;         // work items in flight between roles
+// Consumers of a scheduled item id: the MMA warp and the 8 softmax warps.
+constexpr int kSchedConsumers = 9;
 // Register split.  Launch: 384 threads x 168 = 64512 registers.  After the
 // split: 2 softmax warpgroups x 128 x 208 + 1 control warpgroup x 128 x 88
 // = 53248 + 11264 = 64512, the same total.
@@ -55,9 +64,6 @@ constexpr uint32_t kRegsSoftmax = 208;
 constexpr uint32_t kRegsControl = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
-constexpr int kTmemCols = 512;
-constexpr float kRescaleLog2 = 8.0f;  // rescale O only if max grows > 2^8
-constexpr int kMaxKeyTiles = 256;     // modality mode: Sk <= 32768
 
 template <int D>
 struct FwdCfg {
@@ -70,25 +76,94 @@ struct FwdCfg {
   static constexpr int kSmemK = kTiles * kTileBytes;
   static constexpr int kSmemV = kSmemK + kKStages * kTileBytes;
   static constexpr int kSmemBar = kSmemV + kVStages * kTileBytes;
-  // q_full[2], k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], s_full[2],
-  // p_full[2], o_final[2], drain
-  static constexpr int kNumBars = 2 + 2 * kKStages + 2 * kVStages + 2 + 2 + 2 + 1;
+  // q_full[2], q_empty[2], k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
+  // s_full[2], p_full[2], o_final[2], o_empty[2], drain, sched_full[R],
+  // sched_empty[R]
+  static constexpr int kNumBars = 4 + 2 * kKStages + 2 * kVStages + 8 + 1 + 2 * kSchedRing;
   static constexpr int kSmemMisc = kSmemBar + kNumBars * 8;  // tmem addr, abort
-  static constexpr int kSmemKtBits = kSmemMisc + 16;  // [kt][4] id==1 bits of keys
-  static constexpr int kSmemBytes = kSmemKtBits + kMaxKeyTiles * 16 + 1024;
+  static constexpr int kSmemSched = kSmemMisc + 16;           // int[kSchedRing]
+  static constexpr int kSmemBytes = kSmemSched + 4 * kSchedRing + 1024;
 };
 
-struct TileCtx {
+// One work item: two query tiles of one (b, h).
+struct Item {
   int b, h;
   int q0[kTiles], q_last[kTiles];  // q_last < q0 when the tile has no row
   int nkeys;                       // keys allowed by padding / Sk
   int kt_end;                      // one past the last key tile worth visiting
-  uint32_t q_id_set[kTiles];       // modality: bit a set if some row has id a
+  uint32_t q_ids[kTiles];          // modality: bit a set if some row has id a
 };
 
+__device__ __forceinline__ bool has_rows(const Item& c, int t) {
+  return c.q_last[t] >= c.q0[t];
+}
+
+// Work item number idx of the claim order.  Heads are taken in groups of
+// `group` heads (sized so that their K and V stay in L2 together); within a
+// group, query blocks go longest first under the causal mask (all heads'
+// last block, then the block before, ...).  CTAs claim items dynamically,
+// so long and short items balance out.
+__device__ __forceinline__ Item make_item(const Problem& p, int idx, int q_blocks,
+                                          int group, bool causal) {
+  Item c;
+  const int bn = p.B * p.N;
+  const int per_group = group * q_blocks;
+  const int g = idx / per_group;
+  const int g_heads = min(group, bn - g * group);
+  const int r = idx - g * per_group;
+  const int band = r / g_heads;
+  const int bh = g * group + (r - band * g_heads);
+  const int qb = causal ? (q_blocks - 1 - band) : band;
+  c.b = bh / p.N;
+  c.h = bh - c.b * p.N;
+  c.nkeys = visible_keys(p, c.b);
+  c.kt_end = 0;
+#pragma unroll
+  for (int t = 0; t < kTiles; ++t) {
+    c.q0[t] = qb * kRows + t * kBM;
+    c.q_last[t] = min(c.q0[t] + kBM, p.Sq) - 1;
+    c.q_ids[t] = 0;
+    if (has_rows(c, t)) {
+      int e = (c.nkeys + kBN - 1) / kBN;
+      if (causal) e = min(e, c.q_last[t] / kBN + 1);
+      c.kt_end = max(c.kt_end, e);
+    }
+  }
+  return c;
+}
+
+// Warp-collective: id set (bit a: some position has id a) of ids[lo..hi].
+__device__ __forceinline__ uint32_t warp_id_set(const int32_t* ids, int lo, int hi) {
+  const int lane = threadIdx.x & 31;
+  uint32_t any0 = 0, any1 = 0;
+  for (int base = lo; base <= hi; base += 32) {
+    const int i = base + lane;
+    const bool in = i <= hi;
+    const int id = in ? (ids[i] & 1) : 0;
+    any0 |= __ballot_sync(~0u, in && id == 0);
+    any1 |= __ballot_sync(~0u, in && id == 1);
+  }
+  return (any0 ? 1u : 0u) | (any1 ? 2u : 0u);
+}
+
+// Warp-collective: the modality id sets of the item's query tiles.
+__device__ __forceinline__ void item_query_ids(const Problem& p, Item& c) {
+  if (!(p.mask_flags & FA_MASK_MODALITY)) return;
+  const int32_t* ids = p.ids + int64_t(c.b) * p.Sk;
+#pragma unroll
+  for (int t = 0; t < kTiles; ++t)
+    c.q_ids[t] = has_rows(c, t) ? warp_id_set(ids, c.q0[t], c.q_last[t]) : 0u;
+}
+
+// Warp-collective: id set of key tile kt (modality masks only).
+__device__ __forceinline__ uint32_t key_tile_ids(const Problem& p, const Item& c, int kt) {
+  if (!(p.mask_flags & FA_MASK_MODALITY)) return 0u;
+  return warp_id_set(p.ids + int64_t(c.b) * p.Sk, kt * kBN, min(kt * kBN + kBN, p.Sk) - 1);
+}
+
 // 0 = nothing visible, 1 = partly visible (mask per element), 2 = all visible.
-__device__ __forceinline__ int tile_class(const Problem& p, const TileCtx& c,
-                                          int t, int kt, const uint32_t* kt_bits) {
+__device__ __forceinline__ int tile_class(const Problem& p, const Item& c, int t,
+                                          int kt, uint32_t k_ids) {
   const int q0 = c.q0[t], q_last = c.q_last[t];
   if (q_last < q0) return 0;
   const int k0 = kt * kBN;
@@ -112,22 +187,12 @@ __device__ __forceinline__ int tile_class(const Problem& p, const TileCtx& c,
     }
   }
   if (p.mask_flags & FA_MASK_MODALITY) {
-    // id set of the key tile from its id==1 bits and its valid keys
-    const uint32_t* kb = kt_bits + kt * 4;
-    const int nvalid = min(kBN, p.Sk - k0);
-    uint32_t any1 = 0, any0 = 0;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-      any1 |= kb[w];
-      any0 |= range_bits(0, nvalid - 1, w) & ~kb[w];
-    }
-    const uint32_t ks = (any0 ? 1u : 0u) | (any1 ? 2u : 0u);
     bool any = false, all = true;
 #pragma unroll
     for (int a = 0; a < 2; ++a)
 #pragma unroll
       for (int e = 0; e < 2; ++e)
-        if (((c.q_id_set[t] >> a) & 1u) && ((ks >> e) & 1u)) {
+        if (((c.q_ids[t] >> a) & 1u) && ((k_ids >> e) & 1u)) {
           const bool ok = (p.allow_bits >> (a * 2 + e)) & 1u;
           any |= ok;
           all &= ok;
@@ -145,7 +210,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const Problem p,
                    __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                   int q_blocks) {
+                   int q_blocks, int n_items, int group,
+                   unsigned int* __restrict__ sched) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -155,48 +221,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = smem + C::kSmemV;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
   uint64_t* q_full = bars;
-  uint64_t* k_full = q_full + kTiles;
+  uint64_t* q_empty = q_full + kTiles;
+  uint64_t* k_full = q_empty + kTiles;
   uint64_t* k_empty = k_full + C::kKStages;
   uint64_t* v_full = k_empty + C::kKStages;
   uint64_t* v_empty = v_full + C::kVStages;
   uint64_t* s_full = v_empty + C::kVStages;
   uint64_t* p_full = s_full + kTiles;
   uint64_t* o_final = p_full + kTiles;
-  uint64_t* drain = o_final + kTiles;
+  uint64_t* o_empty = o_final + kTiles;
+  uint64_t* drain = o_empty + kTiles;
+  uint64_t* sched_full = drain + 1;
+  uint64_t* sched_empty = sched_full + kSchedRing;
+  volatile int* sched_ids = reinterpret_cast<volatile int*>(smem + C::kSmemSched);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kSmemMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kSmemMisc + 4);
-  uint32_t* kt_bits = reinterpret_cast<uint32_t*>(smem + C::kSmemKtBits);
 
   const int warp = threadIdx.x >> 5;
   const int tid = threadIdx.x;
+  const int lane = tid & 31;
   const bool causal = p.mask_flags & FA_MASK_CAUSAL;
+  const bool bsh = p.layout == FA_LAYOUT_BSH;
 
-  TileCtx c;
-  c.b = blockIdx.z;
-  c.h = blockIdx.y;
-  // Causal: the longest query blocks first.
-  const int qb = causal ? (q_blocks - 1 - int(blockIdx.x)) : int(blockIdx.x);
-  c.nkeys = visible_keys(p, c.b);
-  c.kt_end = 0;
-#pragma unroll
-  for (int t = 0; t < kTiles; ++t) {
-    c.q0[t] = qb * kRows + t * kBM;
-    c.q_last[t] = min(c.q0[t] + kBM, p.Sq) - 1;
-    c.q_id_set[t] = 0;
-    if (c.q_last[t] >= c.q0[t]) {
-      int e = (c.nkeys + kBN - 1) / kBN;
-      if (causal) e = min(e, c.q_last[t] / kBN + 1);
-      c.kt_end = max(c.kt_end, e);
-    }
-  }
-
-  // ---- set-up: barriers, TMEM, modality id sets
   if (tid == 0) {
     for (int t = 0; t < kTiles; ++t) {
       mbar_init(&q_full[t], 1);
+      mbar_init(&q_empty[t], 1);
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 128);
       mbar_init(&o_final[t], 1);
+      mbar_init(&o_empty[t], 128);
     }
     for (int s = 0; s < C::kKStages; ++s) {
       mbar_init(&k_full[s], 1);
@@ -207,25 +261,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_empty[s], 1);
     }
     mbar_init(drain, 1);
+    for (int s = 0; s < kSchedRing; ++s) {
+      mbar_init(&sched_full[s], 1);
+      mbar_init(&sched_empty[s], kSchedConsumers);
+    }
     *abort_flag = 0;
     fence_barrier_init();
-  }
-  if (p.mask_flags & FA_MASK_MODALITY) {
-    // Per key tile: which ids occur (kt_bits) and the id==1 bits of its keys.
-    const int32_t* ids = p.ids + int64_t(c.b) * p.Sk;
-    const int lane = tid & 31;
-    for (int wk = warp; wk < c.kt_end * 4; wk += kThreads / 32) {
-      const int j = wk * 32 + lane;  // = kt * 128 + w * 32 + lane
-      const bool in = j < p.Sk;
-      const uint32_t is1 = __ballot_sync(~0u, in && (ids[in ? j : 0] & 1) == 1);
-      if (lane == 0) kt_bits[wk] = is1;
-    }
-#pragma unroll
-    for (int t = 0; t < kTiles; ++t) {
-      uint32_t qs = 0;
-      for (int i = c.q0[t] + tid; i <= c.q_last[t]; i += kThreads) qs |= 1u << (ids[i] & 1);
-      c.q_id_set[t] = (__syncthreads_or(qs & 1u) ? 1u : 0u) | (__syncthreads_or(qs & 2u) ? 2u : 0u);
-    }
   }
   if (warp == 9) {
     tmem_alloc(tmem_slot, kTmemCols);
@@ -235,81 +276,122 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const bool bsh = p.layout == FA_LAYOUT_BSH;
-  const int col0 = bsh ? c.h * D : 0;
-  const int z = bsh ? c.b : c.b * p.N + c.h;
+
   if (warp >= 8) {
-   reg_dealloc<kRegsControl>();
-   if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    if (elect_one()) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      if (!(p.debug_flags & 1u)) {  // test hook: never deliver Q
-#pragma unroll
-        for (int t = 0; t < kTiles; ++t) {
-          if (c.q_last[t] < c.q0[t]) continue;
-          mbar_arrive_expect_tx(&q_full[t], C::kTileBytes);
-          for (int x = 0; x < C::kBoxes; ++x)
-            tma_load_3d(sQ + t * C::kTileBytes + x * kBoxBytes, &tm_q, &q_full[t],
-                        col0 + 64 * x, c.q0[t], z);
-        }
+    reg_dealloc<kRegsControl>();
+    if (warp == 8) {
+      // ---------------------------------------------------------- producer
+      // The whole warp walks the schedule (mask classification uses warp
+      // votes); lane 0 issues the copies.
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
       }
       int kidx = 0, vidx = 0;
-      for (int kt = 0; kt < c.kt_end; ++kt) {
-        if (tile_class(p, c, 0, kt, kt_bits) == 0 && tile_class(p, c, 1, kt, kt_bits) == 0)
-          continue;
-        const int sk = kidx % C::kKStages, sv = vidx % C::kVStages;
-        if (kidx >= C::kKStages &&
-            !mbar_wait(&k_empty[sk], ((kidx / C::kKStages) - 1) & 1, abort_flag))
-          break;
-        mbar_arrive_expect_tx(&k_full[sk], C::kTileBytes);
-        for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(sK + sk * C::kTileBytes + x * kBoxBytes, &tm_k, &k_full[sk],
-                      col0 + 64 * x, kt * kBN, z);
-        ++kidx;
-        if (vidx >= C::kVStages &&
-            !mbar_wait(&v_empty[sv], ((vidx / C::kVStages) - 1) & 1, abort_flag))
-          break;
-        mbar_arrive_expect_tx(&v_full[sv], C::kTileBytes);
-        for (int x = 0; x < C::kBoxes; ++x)
-          tma_load_3d(sV + sv * C::kTileBytes + x * kBoxBytes, &tm_v, &v_full[sv],
-                      col0 + 64 * x, kt * kBN, z);
-        ++vidx;
+      int q_uses[kTiles] = {0, 0};
+      bool ok = true;
+      for (int n = 0; ok; ++n) {
+        // Claim the next work item and publish it to the other roles.
+        const int slot = n % kSchedRing;
+        int w = -1;
+        if (lane == 0) {
+          if (n >= kSchedRing &&
+              !mbar_wait(&sched_empty[slot], ((n / kSchedRing) - 1) & 1, abort_flag)) {
+            ok = false;
+          } else {
+            const unsigned int idx = atomicAdd(sched, 1u);
+            w = idx < unsigned(n_items) ? int(idx) : -1;
+            sched_ids[slot] = w;
+            mbar_arrive(&sched_full[slot]);
+          }
+        }
+        ok = __shfl_sync(~0u, ok, 0);
+        w = __shfl_sync(~0u, w, 0);
+        if (!ok || w < 0) break;
+        Item c = make_item(p, w, q_blocks, group, causal);
+        item_query_ids(p, c);
+        const int col0 = bsh ? c.h * D : 0;
+        const int z = bsh ? c.b : c.b * p.N + c.h;
+#pragma unroll
+        for (int t = 0; t < kTiles; ++t) {
+          if (!has_rows(c, t)) continue;
+          if (q_uses[t] > 0) {
+            bool got = true;
+            if (lane == 0) got = mbar_wait(&q_empty[t], (q_uses[t] - 1) & 1, abort_flag);
+            if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
+          }
+          if (lane == 0 && !(p.debug_flags & 1u)) {  // test hook: never deliver Q
+            mbar_arrive_expect_tx(&q_full[t], C::kTileBytes);
+            for (int x = 0; x < C::kBoxes; ++x)
+              tma_load_3d(sQ + t * C::kTileBytes + x * kBoxBytes, &tm_q, &q_full[t],
+                          col0 + 64 * x, c.q0[t], z);
+          }
+          ++q_uses[t];
+        }
+        for (int kt = 0; ok && kt < c.kt_end; ++kt) {
+          const uint32_t kid = key_tile_ids(p, c, kt);
+          if (tile_class(p, c, 0, kt, kid) == 0 && tile_class(p, c, 1, kt, kid) == 0)
+            continue;
+          const int sk = kidx % C::kKStages, sv = vidx % C::kVStages;
+          bool got = true;
+          if (lane == 0 && kidx >= C::kKStages)
+            got = mbar_wait(&k_empty[sk], ((kidx / C::kKStages) - 1) & 1, abort_flag);
+          if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&k_full[sk], C::kTileBytes);
+            for (int x = 0; x < C::kBoxes; ++x)
+              tma_load_3d(sK + sk * C::kTileBytes + x * kBoxBytes, &tm_k, &k_full[sk],
+                          col0 + 64 * x, kt * kBN, z);
+          }
+          ++kidx;
+          if (lane == 0 && vidx >= C::kVStages)
+            got = mbar_wait(&v_empty[sv], ((vidx / C::kVStages) - 1) & 1, abort_flag);
+          if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&v_full[sv], C::kTileBytes);
+            for (int x = 0; x < C::kBoxes; ++x)
+              tma_load_3d(sV + sv * C::kTileBytes + x * kBoxBytes, &tm_v, &v_full[sv],
+                          col0 + 64 * x, kt * kBN, z);
+          }
+          ++vidx;
+        }
       }
-      if (*abort_flag) {
+      if (lane == 0 && *abort_flag) {
         // Let the copies already in flight land before the CTA exits.
         int dummy = 0;
         for (int u = (kidx > C::kKStages ? kidx - C::kKStages : 0); u < kidx; ++u)
           mbar_wait(&k_full[u % C::kKStages], (u / C::kKStages) & 1, &dummy);
         for (int u = (vidx > C::kVStages ? vidx - C::kVStages : 0); u < vidx; ++u)
           mbar_wait(&v_full[u % C::kVStages], (u / C::kVStages) & 1, &dummy);
-        for (int t = 0; t < kTiles; ++t)
-          if (c.q_last[t] >= c.q0[t] && !(p.debug_flags & 1u))
-            mbar_wait(&q_full[t], 0, &dummy);
+        if (!(p.debug_flags & 1u))
+          for (int t = 0; t < kTiles; ++t)
+            if (q_uses[t] > 0) mbar_wait(&q_full[t], (q_uses[t] - 1) & 1, &dummy);
       }
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA
-    if (elect_one()) {
+      __syncwarp();
+    } else if (warp == 9) {
+      // ---------------------------------------------------------- MMA
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
       const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       bool ok = true;
-      bool q_ready[kTiles] = {false, false};
-      int steps[kTiles] = {0, 0};
+      int steps[kTiles] = {0, 0};       // S/P handshakes so far (all items)
       int pend_idx[kTiles] = {-1, -1};  // K/V index whose P V is still to issue
-      int v_users[C::kVStages];
-#pragma unroll
-      for (int s = 0; s < C::kVStages; ++s) v_users[s] = 0;
+      int item_pv[kTiles] = {0, 0};     // P V issued in the current item
+      int o_uses[kTiles] = {0, 0};      // items that produced an O
+      int q_uses[kTiles] = {0, 0};
+      // Outstanding P V per V stage, 4 bits per stage (kept in a register).
+      uint32_t v_users = 0;
 
-      // O_t += P_t V, for the key tile whose S_t the softmax has just turned
+      // O_t += P_t V for the key tile whose S_t the softmax has just turned
       // into P_t.  Issued as soon as P_t is ready so that V stages free up.
+      // Lane 0 only.
       auto issue_pv = [&](int t) -> bool {
         const int vi = pend_idx[t];
         const int sv = vi % C::kVStages;
+        if (item_pv[t] == 0 && o_uses[t] > 0 &&
+            !mbar_wait(&o_empty[t], (o_uses[t] - 1) & 1, abort_flag))
+          return false;  // the previous item's O_t has been read out
         if (!mbar_wait(&p_full[t], (steps[t] - 1) & 1, abort_flag)) return false;
         if (!mbar_wait(&v_full[sv], (vi / C::kVStages) & 1, abort_flag)) return false;
         tc_fence_after();
@@ -318,213 +400,289 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBN / 16; ++kk) {
           const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, kBoxBytes, 1024);
           umma_ts(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8, bdesc, idesc_pv,
-                  (steps[t] > 1 || kk > 0) ? 1u : 0u);
+                  (item_pv[t] > 0 || kk > 0) ? 1u : 0u);
         }
-        if (--v_users[sv] == 0) umma_commit(&v_empty[sv]);
+        v_users -= 1u << (4 * sv);
+        if (((v_users >> (4 * sv)) & 15u) == 0) umma_commit(&v_empty[sv]);
         pend_idx[t] = -1;
+        ++item_pv[t];
         return true;
       };
 
       int idx = 0;
-      for (int kt = 0; ok && kt < c.kt_end; ++kt) {
-        const int cls0 = tile_class(p, c, 0, kt, kt_bits);
-        const int cls1 = tile_class(p, c, 1, kt, kt_bits);
-        if (cls0 == 0 && cls1 == 0) continue;
-        const int sk = idx % C::kKStages;
-        if (!mbar_wait(&k_full[sk], (idx / C::kKStages) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t kbase = sKa + sk * C::kTileBytes;
+      for (int n = 0; ok; ++n) {
+        const int slot = n % kSchedRing;
+        int w = -1;
+        if (lane == 0) {
+          if (mbar_wait(&sched_full[slot], (n / kSchedRing) & 1, abort_flag)) {
+            w = sched_ids[slot];
+            mbar_arrive(&sched_empty[slot]);
+          } else {
+            ok = false;
+          }
+        }
+        ok = __shfl_sync(~0u, ok, 0);
+        w = __shfl_sync(~0u, w, 0);
+        if (!ok || w < 0) break;
+        Item c = make_item(p, w, q_blocks, group, causal);
+        item_query_ids(p, c);
+        // This item's Q tiles (waited even by a tile with no visible key,
+        // so that the phases stay in step with the producer).
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
-          if (pend_idx[t] >= 0 && !issue_pv(t)) { ok = false; break; }
-          if ((t == 0 ? cls0 : cls1) == 0) continue;
-          if (!q_ready[t]) {
-            if (!mbar_wait(&q_full[t], 0, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            q_ready[t] = true;
-          }
-          const uint32_t qbase = sQa + t * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-            umma_ss(tmem + t * 128, sdesc_sw128(qbase + off, 16, 1024),
-                    sdesc_sw128(kbase + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[t]);
-          pend_idx[t] = idx;
-          ++steps[t];
-          ++v_users[idx % C::kVStages];
+          item_pv[t] = 0;
+          if (!has_rows(c, t)) continue;
+          bool got = true;
+          if (lane == 0) got = mbar_wait(&q_full[t], q_uses[t] & 1, abort_flag);
+          if (!__shfl_sync(~0u, got, 0)) ok = false;
+          ++q_uses[t];
         }
         if (!ok) break;
-        umma_commit(&k_empty[sk]);
-        ++idx;
-      }
+        if (lane == 0) tc_fence_after();
+        for (int kt = 0; ok && kt < c.kt_end; ++kt) {
+          const uint32_t kid = key_tile_ids(p, c, kt);
+          const int cls0 = tile_class(p, c, 0, kt, kid);
+          const int cls1 = tile_class(p, c, 1, kt, kid);
+          if (cls0 == 0 && cls1 == 0) continue;
+          if (lane == 0) {
+            const int sk = idx % C::kKStages;
+            if (!mbar_wait(&k_full[sk], (idx / C::kKStages) & 1, abort_flag)) {
+              ok = false;
+            } else {
+              tc_fence_after();
+              const uint32_t kbase = sKa + sk * C::kTileBytes;
 #pragma unroll
-      for (int t = 0; t < kTiles; ++t) {
-        if (ok && pend_idx[t] >= 0 && !issue_pv(t)) ok = false;
-        if (ok && steps[t] > 0) umma_commit(&o_final[t]);
+              for (int t = 0; t < kTiles; ++t) {
+                if (pend_idx[t] >= 0 && !issue_pv(t)) { ok = false; break; }
+                if ((t == 0 ? cls0 : cls1) == 0) continue;
+                const uint32_t qbase = sQa + t * C::kTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
+                  umma_ss(tmem + t * 128, sdesc_sw128(qbase + off, 16, 1024),
+                          sdesc_sw128(kbase + off, 16, 1024), idesc_qk,
+                          kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[t]);
+                pend_idx[t] = idx;
+                ++steps[t];
+                v_users += 1u << (4 * (idx % C::kVStages));
+              }
+              if (ok) umma_commit(&k_empty[sk]);
+            }
+          }
+          ok = __shfl_sync(~0u, ok, 0);
+          ++idx;
+        }
+        if (lane == 0 && ok) {
+#pragma unroll
+          for (int t = 0; t < kTiles; ++t) {
+            if (pend_idx[t] >= 0 && !issue_pv(t)) { ok = false; break; }
+            if (item_pv[t] > 0) {
+              umma_commit(&o_final[t]);
+              ++o_uses[t];
+            }
+            // Q_t may be reloaded once this item's Q K^T are done.
+            if (has_rows(c, t)) umma_commit(&q_empty[t]);
+          }
+        }
+        ok = __shfl_sync(~0u, ok, 0);
       }
-      // Make sure no MMA is in flight when TMEM is released.
-      umma_commit(drain);
-      int dummy = 0;
-      mbar_wait(drain, 0, &dummy);
+      if (lane == 0) {
+        // Make sure no MMA is in flight when TMEM is released.
+        umma_commit(drain);
+        int dummy = 0;
+        mbar_wait(drain, 0, &dummy);
+      }
+      __syncwarp();
     }
-    __syncwarp();
-   }
   } else {
     reg_alloc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;             // query tile of this warpgroup
     const int wq = warp & 3;             // TMEM lane quarter
-    const int row = wq * 32 + (tid & 31);
-    const int i = c.q0[t] + row;         // query index
-    const bool row_real = i < p.Sq;
+    const int row = wq * 32 + lane;
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     const uint32_t tS = tmem + lane_base + t * 128;
     const uint32_t tO = tmem + lane_base + C::kColO + t * D;
     const float sl2 = p.scale_log2;
-    const float slope_l2 = p.slopes ? p.slopes[c.h] * kLog2e : 0.f;
     const bool has_alibi = p.slopes != nullptr;
-    const int32_t* ids = (p.mask_flags & FA_MASK_MODALITY) ? p.ids + int64_t(c.b) * p.Sk : nullptr;
-    const int id_i = (ids && row_real) ? ids[i] : 0;
-    const uint8_t* mrow = (p.mask_flags & FA_MASK_BOOL) && row_real
-                              ? p.mask + c.b * p.m_sb + c.h * p.m_sh + int64_t(i) * p.m_sq
-                              : nullptr;
-
-    float m_ref = -INFINITY;  // reference max (log2 units) of O and l
-    float l = 0.f;
-    int step = 0;
+    int steps = 0, o_uses = 0;
     bool ok = true;
-    const bool tile_has_rows = c.q_last[t] >= c.q0[t];
-    for (int kt = 0; tile_has_rows && kt < c.kt_end; ++kt) {
-      const int cls = tile_class(p, c, t, kt, kt_bits);
-      if (cls == 0) continue;
-      // Every wait is agreed warp-wide before the .sync.aligned TMEM ops.
-      const bool got_s = mbar_wait(&s_full[t], step & 1, abort_flag);
-      if (!__all_sync(~0u, got_s)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, sr[q4]);
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) tmem_ld_wait(sr[q4]);
 
-      // x = s * scale * log2(e) (+ ALiBi), masked -> -inf; kept in sr as fp32.
-      const int k0 = kt * kBN;
-      const uint64_t sl2x2 = f2_pack(sl2, sl2);
-#pragma unroll
-      for (int e = 0; e < 128; e += 2) {
-        float a, b2;
-        f2_unpack(fmul2(f2_pack(__uint_as_float(sr[e >> 5][e & 31]),
-                                __uint_as_float(sr[e >> 5][(e & 31) + 1])),
-                        sl2x2),
-                  a, b2);
-        sr[e >> 5][e & 31] = __float_as_uint(a);
-        sr[e >> 5][(e & 31) + 1] = __float_as_uint(b2);
+    for (int n = 0; ok; ++n) {
+      const int slot = n % kSchedRing;
+      int w = -1;
+      if (lane == 0) {
+        if (mbar_wait(&sched_full[slot], (n / kSchedRing) & 1, abort_flag)) {
+          w = sched_ids[slot];
+          mbar_arrive(&sched_empty[slot]);
+        } else {
+          ok = false;
+        }
       }
-      if (has_alibi) {
+      ok = __shfl_sync(~0u, ok, 0);
+      w = __shfl_sync(~0u, w, 0);
+      if (!ok || w < 0) break;
+      Item c = make_item(p, w, q_blocks, group, causal);
+      item_query_ids(p, c);
+      if (!has_rows(c, t)) continue;
+      const int i = c.q0[t] + row;  // query index
+      const bool row_real = i < p.Sq;
+      const float slope_l2 = has_alibi ? p.slopes[c.h] * kLog2e : 0.f;
+      const int32_t* ids =
+          (p.mask_flags & FA_MASK_MODALITY) ? p.ids + int64_t(c.b) * p.Sk : nullptr;
+      const int id_i = (ids && row_real) ? (ids[i] & 1) : 0;
+      const uint8_t* mrow = (p.mask_flags & FA_MASK_BOOL) && row_real
+                                ? p.mask + c.b * p.m_sb + c.h * p.m_sh + int64_t(i) * p.m_sq
+                                : nullptr;
+      float m_ref = -INFINITY;  // reference max (log2 units) of O and l
+      float l = 0.f;
+      int item_steps = 0;
+
+      for (int kt = 0; kt < c.kt_end; ++kt) {
+        const uint32_t kid = key_tile_ids(p, c, kt);
+        const int cls = tile_class(p, c, t, kt, kid);
+        if (cls == 0) continue;
+        // Every wait is agreed warp-wide before the .sync.aligned TMEM ops.
+        const bool got_s = mbar_wait(&s_full[t], steps & 1, abort_flag);
+        if (!__all_sync(~0u, got_s)) { ok = false; break; }
+        tc_fence_after();
+        const int k0 = kt * kBN;
+        // Without a bias and with a positive scale, max(s * c) = c * max(s)
+        // exactly, and x - m folds into one fma per element; the same
+        // arithmetic is used whether or not the tile needs masking, so the
+        // result does not depend on the tile classification.
+        const bool plain = !has_alibi && sl2 > 0.f;
+        const bool masked = cls == 1;
+        uint32_t sr[4][32];
 #pragma unroll
-        for (int e = 0; e < 128; ++e)
-          sr[e >> 5][e & 31] = __float_as_uint(
-              fmaf(-slope_l2, float(abs(i - (k0 + e))), __uint_as_float(sr[e >> 5][e & 31])));
-      }
-      if (cls == 1) {
-        // Visibility of the 128 keys of this tile for row i, as bits.
-        int lim = row_real ? (c.nkeys - 1 - k0) : -1;  // keys e <= lim visible
-        if (causal) lim = min(lim, i - k0);
-        uint32_t vb[4];
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, sr[q4]);
 #pragma unroll
-        for (int w = 0; w < 4; ++w) vb[w] = range_bits(0, lim, w);
-        if (mrow) {
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld_wait(sr[q4]);
+        if (!plain) {
+          // x = s * scale * log2(e) + ALiBi, kept in sr
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            float x = __uint_as_float(sr[e >> 5][e & 31]) * sl2;
+            if (has_alibi) x = fmaf(-slope_l2, float(abs(i - (k0 + e))), x);
+            sr[e >> 5][e & 31] = __float_as_uint(x);
+          }
+        }
+        if (masked) {
+          // Key ids of this tile as id==1 bits (modality rule), by warp votes.
+          uint32_t kb[4] = {0u, 0u, 0u, 0u};
+          if (ids && cls == 1) {
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+              const int j = k0 + 32 * wd + lane;
+              kb[wd] = __ballot_sync(~0u, j < p.Sk && (ids[j < p.Sk ? j : 0] & 1) == 1);
+            }
+          }
+          // Visibility of the 128 keys of this tile for row i, as bits.
+          uint32_t vb[4];
+          {
+            int lim = row_real ? (c.nkeys - 1 - k0) : -1;  // keys e <= lim visible
+            if (causal) lim = min(lim, i - k0);
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) vb[wd] = range_bits(0, lim, wd);
+            if (mrow) {
 #pragma unroll 1
-          for (int w = 0; w < 4; ++w) {
-            uint32_t m = 0;
-            const int jw = k0 + 32 * w;
-            for (int e = 0; e < 32 && jw + e < p.Sk; ++e) m |= uint32_t(mrow[jw + e] != 0) << e;
-            vb[w] &= m;
+              for (int wd = 0; wd < 4; ++wd) {
+                uint32_t m = 0;
+                const int jw = k0 + 32 * wd;
+                for (int e = 0; e < 32 && jw + e < p.Sk; ++e)
+                  m |= uint32_t(mrow[jw + e] != 0) << e;
+                vb[wd] &= m;
+              }
+            }
+            if (ids) {
+#pragma unroll
+              for (int wd = 0; wd < 4; ++wd) {
+                uint32_t m = modality_row_bits(p.allow_bits, id_i, kb[wd], true);
+                if (p.allow_bits & 16u) m |= range_bits(i - k0, i - k0, wd);
+                vb[wd] &= m;
+              }
+            }
+          }
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (!((vb[e >> 5] >> (e & 31)) & 1u)) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
+        }
+        // Row max with 8 independent chains.
+        float mx8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sr[0][u]);
+#pragma unroll
+        for (int e = 8; e < 128; ++e)
+          mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[e >> 5][e & 31]));
+        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        if (plain) mx *= sl2;  // -inf stays -inf (sl2 > 0)
+        // Move the reference max only when it grew by more than 2^8: O and l
+        // are then rescaled by alpha (exact after the final division).
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mx > m_ref + kRescaleLog2) {  // false while mx = -inf
+          alpha = ex2_approx(m_ref - mx);  // 0 when m_ref = -inf
+          m_ref = mx;
+          rescale = true;
+        }
+        // P = 2^(x - m) in bf16, written over the S columns already read
+        // (keys 32q..32q+31 -> packed columns 16q..16q+15).
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        const uint64_t neg_m = f2_pack(-m_use, -m_use);
+        const uint64_t sl2x2 = f2_pack(sl2, sl2);
+        uint64_t rs2[4] = {0, 0, 0, 0};  // 4 chains of packed partial sums
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const uint64_t s2 = f2_pack(__uint_as_float(sr[q4][e]), __uint_as_float(sr[q4][e + 1]));
+            float a0, a1;
+            f2_unpack(plain ? ffma2(s2, sl2x2, neg_m) : fadd2(s2, neg_m), a0, a1);
+            const float p0 = ex2_approx(a0);  // 2^-inf = 0 for masked keys
+            const float p1 = ex2_approx(a1);
+            rs2[(e >> 1) & 3] = fadd2(rs2[(e >> 1) & 3], f2_pack(p0, p1));
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + q4 * 16, pk);
+        }
+        if (item_steps > 0 && __any_sync(~0u, rescale)) {
+          // S ready implies every earlier MMA (the previous P V) is complete,
+          // and the next P V of this tile waits for P, so O is quiescent.
+          const float a = rescale ? alpha : 1.f;
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t orr[32];
+            tmem_ld32(tO + cc * 32, orr);
+            tmem_ld_wait(orr);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * a);
+            tmem_st32(tO + cc * 32, orr);
           }
         }
-        if (ids) {
-          const uint32_t* kb = kt_bits + kt * 4;
+        float r[8];
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            uint32_t m = modality_row_bits(p.allow_bits, id_i, kb[w], true);
-            if (p.allow_bits & 16u) m |= range_bits(i - k0, i - k0, w);
-            vb[w] &= m;
-          }
-        }
-#pragma unroll
-        for (int e = 0; e < 128; ++e)
-          if (!((vb[e >> 5] >> (e & 31)) & 1u)) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
+        for (int u = 0; u < 4; ++u) f2_unpack(rs2[u], r[2 * u], r[2 * u + 1]);
+        l = l * alpha + (((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7])));
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
+        ++steps;
+        ++item_steps;
       }
-      // Row max with 8 independent chains.
-      float mx8[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sr[0][u]);
-#pragma unroll
-      for (int e = 8; e < 128; ++e)
-        mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[e >> 5][e & 31]));
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-      // Move the reference max only when it grew by more than 2^8: O and l
-      // are then rescaled by alpha (exact after the final division).
-      float alpha = 1.f;
-      bool rescale = false;
-      if (mx > m_ref + kRescaleLog2) {  // false while mx = -inf
-        alpha = ex2_approx(m_ref - mx);  // 0 when m_ref = -inf
-        m_ref = mx;
-        rescale = true;
-      }
-      if (step > 0 && __any_sync(~0u, rescale)) {
-        // S ready implies every earlier MMA (the previous P V) is complete,
-        // and the next P V of this tile waits for P, so O is quiescent.
-        const float a = rescale ? alpha : 1.f;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t orr[32];
-          tmem_ld32(tO + cc * 32, orr);
-          tmem_ld_wait(orr);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * a);
-          tmem_st32(tO + cc * 32, orr);
-        }
-      }
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      const uint64_t neg_m = f2_pack(-m_use, -m_use);
-      uint64_t rs2[4] = {0, 0, 0, 0};  // 4 chains of packed partial sums
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int e = 0; e < 64; e += 2) {
-          const int g = half * 64 + e;
-          float a0, a1;
-          f2_unpack(fadd2(f2_pack(__uint_as_float(sr[g >> 5][g & 31]),
-                                  __uint_as_float(sr[g >> 5][(g & 31) + 1])),
-                          neg_m),
-                    a0, a1);
-          const float p0 = ex2_approx(a0);
-          const float p1 = ex2_approx(a1);
-          rs2[(e >> 1) & 3] = fadd2(rs2[(e >> 1) & 3], f2_pack(p0, p1));
-          pk[e >> 1] = pack_bf16x2(p0, p1);
-        }
-        tmem_st32(tS + half * 32, pk);
-      }
-      float r[8];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) f2_unpack(rs2[u], r[2 * u], r[2 * u + 1]);
-      l = l * alpha + (((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7])));
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-      ++step;
-    }
+      if (!ok) break;
 
-    // ---------------------------------------------------------- epilogue
-    if (tile_has_rows) {
-      const bool have_o =
-          __all_sync(~0u, ok && step > 0 && mbar_wait(&o_final[t], 0, abort_flag));
-      if (have_o) tc_fence_after();
+      // -------------------------------------------------------- epilogue
+      bool have_o = false;
+      if (item_steps > 0) {
+        have_o = __all_sync(~0u, mbar_wait(&o_final[t], o_uses & 1, abort_flag));
+        if (!have_o) { ok = false; break; }
+        ++o_uses;
+        tc_fence_after();
+      }
       const bool empty = !(l > 0.f);
       const float inv = empty ? 0.f : 1.f / l;
       __nv_bfloat16* orow = out + c.b * p.q_sb + c.h * p.q_sh + int64_t(i) * p.q_ss;
@@ -534,19 +692,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (have_o) {
           tmem_ld32(tO + cc * 32, orr);
           tmem_ld_wait(orr);
+          if (cc == D / 32 - 1) {
+            // O_t has been read: the next item's first P V may overwrite it.
+            tc_fence_before();
+            mbar_arrive(&o_empty[t]);
+          }
         }
         if (row_real) {
-          uint32_t w[16];
+          uint32_t wv[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const float o0 = (have_o && !empty) ? __uint_as_float(orr[2 * e]) * inv : 0.f;
             const float o1 = (have_o && !empty) ? __uint_as_float(orr[2 * e + 1]) * inv : 0.f;
-            w[e] = pack_bf16x2(o0, o1);
+            wv[e] = pack_bf16x2(o0, o1);
           }
           uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
         }
       }
       if (row_real)
@@ -562,6 +725,38 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_dealloc(tmem, kTmemCols);
   }
   if (tid == 0 && *abort_flag) atomicOr(p.status, 1u);
+}
+
+// Work-item counters for the dynamic scheduler, one per launch in flight
+// (a launch takes the next slot and clears it on its stream first).
+constexpr int kSchedSlots = 64;
+__device__ unsigned int g_fwd_sched[kSchedSlots];
+
+unsigned int* sched_slot() {
+  static unsigned int* base[64] = {};
+  static unsigned int ticket = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!base[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_fwd_sched) != cudaSuccess) return nullptr;
+    base[dev] = static_cast<unsigned int*>(a);
+  }
+  const unsigned int t = __atomic_fetch_add(&ticket, 1u, __ATOMIC_RELAXED);
+  return base[dev] + (t % kSchedSlots);
+}
+
+int sm_count() {
+  static int count[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (count[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    count[dev] = n;
+  }
+  return count[dev];
 }
 
 }  // namespace
@@ -581,9 +776,21 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
                            C::kSmemBytes);
   if (e != cudaSuccess) return e;
   const int q_blocks = (p.Sq + kRows - 1) / kRows;
-  dim3 grid(q_blocks, p.N, p.B);
+  const int64_t items = int64_t(q_blocks) * p.B * p.N;
+  if (items > 0x7fffffff) return cudaErrorInvalidValue;
+  const int grid = int(items < sm_count() ? items : sm_count());
+  // Heads per scheduling group: about one L2 (126 MB) of K and V.  Larger
+  // groups give the longest-first order more room; smaller ones keep the
+  // K/V tiles of concurrently processed items resident.
+  const int64_t kv_bytes = int64_t(2) * p.Sk * p.D * 2;
+  int group = int((int64_t(128) << 20) / (kv_bytes > 0 ? kv_bytes : 1));
+  group = group < 1 ? 1 : (group > p.B * p.N ? p.B * p.N : group);
+  unsigned int* sched = sched_slot();
+  if (!sched) return cudaErrorUnknown;
+  if ((e = cudaMemsetAsync(sched, 0, sizeof(unsigned int), st)) != cudaSuccess) return e;
   fwd_bf16_sm100<D><<<grid, kThreads, C::kSmemBytes, st>>>(
-      tq, tk, tv, p, static_cast<__nv_bfloat16*>(out), lse, q_blocks);
+      tq, tk, tv, p, static_cast<__nv_bfloat16*>(out), lse, q_blocks, int(items), group,
+      sched);
   return cudaGetLastError();
 }
 
