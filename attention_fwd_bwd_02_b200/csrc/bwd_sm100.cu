@@ -9,19 +9,23 @@
 //
 // One CTA owns a 128-key tile of one (b, h) and walks the 64-row query tiles
 // that can see it.  Everything is computed transposed, keys on the TMEM
-// lanes:
-//   S^T  = K Q^T      (SS)            -> TMEM cols [0, 64)
-//   dP^T = V dO^T     (SS)            -> TMEM cols [64, 128)
-//   P^T, dS^T (bf16) written back over S^T and dP^T by the softmax warps
-//   dV  += P^T dO     (P^T from TMEM) -> TMEM cols [128, 128+D)
-//   dK  += dS^T Q     (dS^T from TMEM)-> TMEM cols [128+D, 128+2D)
-//   dQ^T = K^T dS^T   (SS, dS^T staged in shared memory)
-//                                     -> TMEM cols [128+2D, 128+2D+64)
-// dQ^T of each query tile is read by a dedicated warpgroup, staged in
-// shared memory and added to the fp32 dQ accumulator in global memory with
-// one bulk reduce-add per tile.
-// Warp roles: 0-3 softmax (thread = key row) and the dK/dV epilogue,
-// 4-7 dQ reduction, 8 TMA producer, 9 MMA issuer and TMEM owner.
+// lanes.  Two TMEM buffers of 128 columns alternate between query tiles:
+//   S^T = K Q^T  (SS) -> cols [0, 64),  dP^T = V dO^T (SS) -> cols [64, 128)
+//   the softmax warps then write P^T (bf16) to cols [0, 32) and dS^T (bf16)
+//   to cols [32, 64), and dQ^T = K^T dS^T (SS, dS^T staged in shared memory)
+//   lands in cols [64, 128).
+//   dV += P^T dO  (P^T from TMEM) and dK += dS^T Q (dS^T from TMEM)
+//   accumulate in cols [256, 256+D) and [256+D, 256+2D).
+// dQ^T of each query tile is read by a dedicated warpgroup, staged in shared
+// memory and added to the fp32 dQ accumulator in global memory with tiled
+// TMA reduce-adds (one per warp and tile).
+// Warp roles (16 warps):
+//   0-3 / 4-7  softmax of even / odd query tiles (thread = key row), and the
+//              dK / dV epilogue (warps 0-3 write dV, warps 4-7 write dK);
+//   8-11       dQ reduction;
+//   12         TMA producer;  13  MMA issuer and TMEM owner;  14-15 idle.
+// While one softmax warpgroup works on query tile n, the tensor core runs the
+// MMAs of tiles n-1 and n+1 and the other warpgroup works on tile n+1.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -37,50 +41,54 @@ namespace {
 
 constexpr int kBN = 128;  // keys per CTA
 constexpr int kBM = 64;   // query rows per step
-constexpr int kThreads = 320;
+constexpr int kThreads = 512;
 constexpr int kTmemCols = 512;
 constexpr int kKeyBox = 128 * 128;  // 128 rows x 64 cols bf16
 constexpr int kQBox = 64 * 128;     // 64 rows x 64 cols bf16
-constexpr int kMaxQTiles = 512;     // modality mode: Sq <= 32768
-constexpr int kColS = 0, kColDP = 64, kColDV = 128;
+constexpr int kColP = 0, kColDS = 32, kColDQ = 64, kColAcc = 256;
+// Register split.  Launch: 512 threads x 128 = 65536 registers.  After the
+// split: 2 softmax warpgroups x 128 x 168 + dQ warpgroup x 128 x 88 + control
+// warpgroup x 128 x 88 = 43008 + 11264 + 11264 = 65536.
+constexpr uint32_t kRegsSoftmax = 168;
+constexpr uint32_t kRegsDq = 88;
+constexpr uint32_t kRegsControl = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsDq + 128 * kRegsControl <= 65536,
+              "register split exceeds the launch allocation");
 
 template <int D>
 struct BwdCfg {
   static constexpr int kBoxes = D / 64;
   static constexpr int kKTile = kBoxes * kKeyBox;  // 128 keys x D
   static constexpr int kQTile = kBoxes * kQBox;    // 64 rows x D
-  static constexpr int kStages = 2;
-  static constexpr int kColDK = kColDV + D;
-  static constexpr int kColDQ = kColDV + 2 * D;
+  static constexpr int kStages = 3;                // Q / dO ring
+  static constexpr int kColDV = kColAcc;
+  static constexpr int kColDK = kColAcc + D;
   static constexpr int kSmemK = 0;
   static constexpr int kSmemV = kSmemK + kKTile;
   static constexpr int kSmemQ = kSmemV + kKTile;                 // [stage]
   static constexpr int kSmemDO = kSmemQ + kStages * kQTile;      // [stage]
-  static constexpr int kSmemDS = kSmemDO + kStages * kQTile;     // 128 x 64 bf16
-  // dQ staging: per dQ warp, 2 buffers of 64 rows x (D / 4) fp32 columns
+  static constexpr int kSmemDS = kSmemDO + kStages * kQTile;     // [2] 128 x 64 bf16
+  // dQ staging: per dQ warp one box of 64 rows x (D / 4) fp32 columns
   static constexpr int kDqCols = D / 4;
   static constexpr int kStageBytes = kBM * kDqCols * 4;
-  static constexpr int kSmemStage = kSmemDS + 128 * 128;
-  static constexpr int kSmemStats = kSmemStage + 4 * 2 * kStageBytes;  // [4 warps][2][64] fp32
-  static constexpr int kSmemBar = kSmemStats + 4 * 2 * kBM * 4;
-  // kv_full, q_full[S], q_empty[S], s_full, p_ready, ds_free, dq_full,
-  // dq_free, acc_done, drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 7;
+  static constexpr int kSmemStage = kSmemDS + 2 * 128 * 128;
+  static constexpr int kSmemBar = kSmemStage + 4 * kStageBytes;
+  // kv_full, q_full[3], q_empty[3], s_full[2], p_ready[2], dq_full[2],
+  // dq_free[2], acc_done, drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 8 + 2;
   static constexpr int kSmemMisc = kSmemBar + kNumBars * 8;
-  static constexpr int kSmemQtBits = kSmemMisc + 16;  // [qt][2] id==1 bits of queries
-  static constexpr int kSmemBytes = kSmemQtBits + kMaxQTiles * 8 + 1024;
+  static constexpr int kSmemBytes = kSmemMisc + 16 + 1024;
 };
 
 struct KeyCtx {
   int b, h, k0, k_last;  // k_last = last key of the tile inside Sk
   int nkeys;             // visible keys of batch b (padding rule)
   int qt_begin, qt_end;  // query tiles (of 64) worth visiting
-  uint32_t k_id_set;     // modality: id set of the tile's keys
 };
 
 // 0 = no visible pair, 1 = some pairs (mask per element), 2 = all pairs.
-__device__ __forceinline__ int qtile_class(const Problem& p, const KeyCtx& c,
-                                           int qt, const uint32_t* qt_bits) {
+// Modality masks are always treated as partly visible here.
+__device__ __forceinline__ int qtile_class(const Problem& p, const KeyCtx& c, int qt) {
   const int q0 = qt * kBM;
   const int q_last = min(q0 + kBM, p.Sq) - 1;
   if (c.k0 >= c.nkeys) return 0;
@@ -102,31 +110,26 @@ __device__ __forceinline__ int qtile_class(const Problem& p, const KeyCtx& c,
       cls = 1;
     }
   }
-  if (p.mask_flags & FA_MASK_MODALITY) {
-    // id set of the query tile from its id==1 bits and its valid rows
-    const int nvalid = min(kBM, p.Sq - q0);
-    uint32_t any1 = 0, any0 = 0;
-#pragma unroll
-    for (int w = 0; w < 2; ++w) {
-      any1 |= qt_bits[qt * 2 + w];
-      any0 |= range_bits(0, nvalid - 1, w) & ~qt_bits[qt * 2 + w];
-    }
-    const uint32_t qs = (any0 ? 1u : 0u) | (any1 ? 2u : 0u);
-    bool any = false, all = true;
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int e = 0; e < 2; ++e)
-        if (((qs >> a) & 1u) && ((c.k_id_set >> e) & 1u)) {
-          const bool ok = (p.allow_bits >> (a * 2 + e)) & 1u;
-          any |= ok;
-          all &= ok;
-        }
-    const bool diag = (p.allow_bits & 16u) && (c.k0 <= q_last) && (q0 <= c.k_last);
-    if (!any && !diag) return 0;
-    if (!all) cls = 1;
-  }
+  if (p.mask_flags & FA_MASK_MODALITY) cls = 1;
   return cls;
+}
+
+// Number of query tiles visited before qt (the step index of qt).
+template <typename F>
+__device__ __forceinline__ void for_each_qtile(const Problem& p, const KeyCtx& c, F f) {
+  int n = 0;
+  for (int qt = c.qt_begin; qt < c.qt_end; ++qt) {
+    const int cls = qtile_class(p, c, qt);
+    if (cls == 0) continue;
+    if (!f(n, qt, cls)) return;
+    ++n;
+  }
+}
+
+__device__ __forceinline__ int count_qtiles(const Problem& p, const KeyCtx& c) {
+  int n = 0;
+  for (int qt = c.qt_begin; qt < c.qt_end; ++qt) n += qtile_class(p, c, qt) != 0;
+  return n;
 }
 
 // First dQ column owned by dQ warp wq.
@@ -140,8 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_dq, const Problem p,
                    const float* __restrict__ lse, const float* __restrict__ delta,
-                   float* __restrict__ dq_acc, __nv_bfloat16* __restrict__ dk,
-                   __nv_bfloat16* __restrict__ dv) {
+                   __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -152,21 +154,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sDO = smem + C::kSmemDO;
   uint8_t* sDS = smem + C::kSmemDS;
   float* sStage = reinterpret_cast<float*>(smem + C::kSmemStage);
-  float* sStats = reinterpret_cast<float*>(smem + C::kSmemStats);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;
   uint64_t* q_empty = q_full + C::kStages;
   uint64_t* s_full = q_empty + C::kStages;
-  uint64_t* p_ready = s_full + 1;
-  uint64_t* ds_free = p_ready + 1;
-  uint64_t* dq_full = ds_free + 1;
-  uint64_t* dq_free = dq_full + 1;
-  uint64_t* acc_done = dq_free + 1;
+  uint64_t* p_ready = s_full + 2;
+  uint64_t* dq_full = p_ready + 2;
+  uint64_t* dq_free = dq_full + 2;
+  uint64_t* acc_done = dq_free + 2;
   uint64_t* drain = acc_done + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kSmemMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kSmemMisc + 4);
-  uint32_t* qt_bits = reinterpret_cast<uint32_t*>(smem + C::kSmemQtBits);
 
   const int warp = threadIdx.x >> 5;
   const int tid = threadIdx.x;
@@ -180,7 +179,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.nkeys = visible_keys(p, c.b);
   c.qt_begin = (p.mask_flags & FA_MASK_CAUSAL) ? c.k0 / kBM : 0;
   c.qt_end = (p.Sq + kBM - 1) / kBM;
-  c.k_id_set = 0;
 
   if (tid == 0) {
     mbar_init(kv_full, 1);
@@ -188,29 +186,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_ready, 128);
-    mbar_init(ds_free, 1);
-    mbar_init(dq_full, 1);
-    mbar_init(dq_free, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_ready[b], 128);
+      mbar_init(&dq_full[b], 1);
+      mbar_init(&dq_free[b], 128);
+    }
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (p.mask_flags & FA_MASK_MODALITY) {
-    const int32_t* ids = p.ids + int64_t(c.b) * p.Sk;
-    for (int wq = c.qt_begin * 2 + warp; wq < c.qt_end * 2; wq += kThreads / 32) {
-      const int i = wq * 32 + lane;  // = qt * 64 + w * 32 + lane
-      const bool in = i < p.Sq;
-      const uint32_t is1 = __ballot_sync(~0u, in && (ids[in ? i : 0] & 1) == 1);
-      if (lane == 0) qt_bits[wq] = is1;
-    }
-    uint32_t ks = 0;
-    for (int j = c.k0 + tid; j <= c.k_last; j += kThreads) ks |= 1u << (ids[j] & 1);
-    c.k_id_set = __syncthreads_or(ks & 1u) | (__syncthreads_or(ks & 2u) ? 2u : 0u);
-  }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -219,126 +206,138 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool bsh = p.layout == FA_LAYOUT_BSH;
-  const int col0 = bsh ? c.h * D : 0;
-  const int z = bsh ? c.b : c.b * p.N + c.h;
 
-  if (warp == 8) {
-    // ------------------------------------------------------------ producer
-    if (elect_one()) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_do);
-      mbar_arrive_expect_tx(kv_full, 2 * C::kKTile);
-      for (int x = 0; x < C::kBoxes; ++x) {
-        tma_load_3d(sK + x * kKeyBox, &tm_k, kv_full, col0 + 64 * x, c.k0, z);
-        tma_load_3d(sV + x * kKeyBox, &tm_v, kv_full, col0 + 64 * x, c.k0, z);
-      }
-      int n = 0;
-      for (int qt = c.qt_begin; qt < c.qt_end; ++qt) {
-        if (qtile_class(p, c, qt, qt_bits) == 0) continue;
-        const int st = n % C::kStages, use = n / C::kStages;
-        if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&q_full[st], 2 * C::kQTile);
+  if (warp >= 12) {
+    reg_dealloc<kRegsControl>();
+    const int col0 = bsh ? c.h * D : 0;
+    const int z = bsh ? c.b : c.b * p.N + c.h;
+    if (warp == 12) {
+      // ---------------------------------------------------------- producer
+      if (elect_one()) {
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_do);
+        mbar_arrive_expect_tx(kv_full, 2 * C::kKTile);
         for (int x = 0; x < C::kBoxes; ++x) {
-          tma_load_3d(sQ + st * C::kQTile + x * kQBox, &tm_q, &q_full[st],
-                      col0 + 64 * x, qt * kBM, z);
-          tma_load_3d(sDO + st * C::kQTile + x * kQBox, &tm_do, &q_full[st],
-                      col0 + 64 * x, qt * kBM, z);
+          tma_load_3d(sK + x * kKeyBox, &tm_k, kv_full, col0 + 64 * x, c.k0, z);
+          tma_load_3d(sV + x * kKeyBox, &tm_v, kv_full, col0 + 64 * x, c.k0, z);
         }
-        ++n;
+        int issued = 0;
+        for_each_qtile(p, c, [&](int n, int qt, int) -> bool {
+          const int st = n % C::kStages, use = n / C::kStages;
+          if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, abort_flag)) return false;
+          mbar_arrive_expect_tx(&q_full[st], 2 * C::kQTile);
+          for (int x = 0; x < C::kBoxes; ++x) {
+            tma_load_3d(sQ + st * C::kQTile + x * kQBox, &tm_q, &q_full[st],
+                        col0 + 64 * x, qt * kBM, z);
+            tma_load_3d(sDO + st * C::kQTile + x * kQBox, &tm_do, &q_full[st],
+                        col0 + 64 * x, qt * kBM, z);
+          }
+          issued = n + 1;
+          return true;
+        });
+        // Let every copy this thread issued land before the CTA can exit.
+        int dummy = 0;
+        mbar_wait(kv_full, 0, &dummy);
+        const int first = issued > C::kStages ? issued - C::kStages : 0;
+        for (int u = first; u < issued; ++u)
+          mbar_wait(&q_full[u % C::kStages], (u / C::kStages) & 1, &dummy);
       }
-      // Let every copy this thread issued land before the CTA can exit.
-      int dummy = 0;
-      mbar_wait(kv_full, 0, &dummy);
-      const int first = n > C::kStages ? n - C::kStages : 0;
-      for (int u = first; u < n; ++u)
-        mbar_wait(&q_full[u % C::kStages], (u / C::kStages) & 1, &dummy);
-    }
-    __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA
-    if (elect_one()) {
-      constexpr uint32_t id_s = idesc_bf16_f32(128, kBM, 0, 0);   // S^T, dP^T
-      constexpr uint32_t id_kv = idesc_bf16_f32(128, D, 0, 1);    // dV, dK
-      constexpr uint32_t id_q = idesc_bf16_f32(D, kBM, 1, 1);     // dQ^T
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
-      const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aDS = smem_u32(sDS);
-      bool ok = mbar_wait(kv_full, 0, abort_flag);
-      int n = 0;
-      for (int qt = c.qt_begin; ok && qt < c.qt_end; ++qt) {
-        if (qtile_class(p, c, qt, qt_bits) == 0) continue;
-        const int st = n % C::kStages;
-        if (!mbar_wait(&q_full[st], (n / C::kStages) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t q_base = aQ + st * C::kQTile, do_base = aDO + st * C::kQTile;
-        // S^T = K Q^T and dP^T = V dO^T
+      __syncwarp();
+    } else if (warp == 13) {
+      // ---------------------------------------------------------- MMA
+      if (elect_one()) {
+        constexpr uint32_t id_s = idesc_bf16_f32(128, kBM, 0, 0);  // S^T, dP^T
+        constexpr uint32_t id_kv = idesc_bf16_f32(128, D, 0, 1);   // dV, dK
+        constexpr uint32_t id_q = idesc_bf16_f32(D, kBM, 1, 1);    // dQ^T
+        const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
+        const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aDS = smem_u32(sDS);
+        const int n_tiles = count_qtiles(p, c);
+        bool ok = mbar_wait(kv_full, 0, abort_flag);
+        // S^T = K Q^T and dP^T = V dO^T of step n into buffer n % 2.
+        auto issue_sdp = [&](int n) -> bool {
+          const int st = n % C::kStages, b = n & 1;
+          if (!mbar_wait(&q_full[st], (n / C::kStages) & 1, abort_flag)) return false;
+          tc_fence_after();
+          const uint32_t q_base = aQ + st * C::kQTile, do_base = aDO + st * C::kQTile;
+          const uint32_t tb = tmem + b * 128;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ko = (kk >> 2) * kKeyBox + (kk & 3) * 32;
-          const uint32_t qo = (kk >> 2) * kQBox + (kk & 3) * 32;
-          umma_ss(tmem + kColS, sdesc_sw128(aK + ko, 16, 1024),
-                  sdesc_sw128(q_base + qo, 16, 1024), id_s, kk > 0 ? 1u : 0u);
-          umma_ss(tmem + kColDP, sdesc_sw128(aV + ko, 16, 1024),
-                  sdesc_sw128(do_base + qo, 16, 1024), id_s, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full);
-        if (!mbar_wait(p_ready, n & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        // dV += P^T dO ; dK += dS^T Q   (A operands from TMEM)
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ko = (kk >> 2) * kKeyBox + (kk & 3) * 32;
+            const uint32_t qo = (kk >> 2) * kQBox + (kk & 3) * 32;
+            umma_ss(tb, sdesc_sw128(aK + ko, 16, 1024), sdesc_sw128(q_base + qo, 16, 1024),
+                    id_s, kk > 0 ? 1u : 0u);
+            umma_ss(tb + 64, sdesc_sw128(aV + ko, 16, 1024),
+                    sdesc_sw128(do_base + qo, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[b]);
+          return true;
+        };
+        if (ok && n_tiles > 0) ok = issue_sdp(0);
+        if (ok && n_tiles > 1) ok = issue_sdp(1);
+        for (int n = 0; ok && n < n_tiles; ++n) {
+          const int st = n % C::kStages, b = n & 1;
+          const uint32_t tb = tmem + b * 128;
+          if (!mbar_wait(&p_ready[b], (n >> 1) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          // dQ^T = K^T dS^T first, so that its read-out overlaps dV and dK.
 #pragma unroll
-        for (int kk = 0; kk < kBM / 16; ++kk) {
-          const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-          umma_ts(tmem + kColDV, tmem + kColS + kk * 8,
-                  sdesc_sw128(do_base + kk * 2048, kQBox, 1024), id_kv, acc);
-          umma_ts(tmem + C::kColDK, tmem + kColDP + kk * 8,
-                  sdesc_sw128(q_base + kk * 2048, kQBox, 1024), id_kv, acc);
-        }
-        umma_commit(&q_empty[st]);
-        // dQ^T = K^T dS^T once the previous dQ^T has been read out
-        if (n > 0 && !mbar_wait(dq_free, (n - 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            umma_ss(tb + kColDQ, sdesc_sw128(aK + kk * 2048, kKeyBox, 1024),
+                    sdesc_sw128(aDS + b * 16384 + kk * 2048, kKeyBox, 1024), id_q,
+                    kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&dq_full[b]);
+          // dV += P^T dO ; dK += dS^T Q   (A operands from TMEM)
+          const uint32_t q_base = aQ + st * C::kQTile, do_base = aDO + st * C::kQTile;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          umma_ss(tmem + C::kColDQ, sdesc_sw128(aK + kk * 2048, kKeyBox, 1024),
-                  sdesc_sw128(aDS + kk * 2048, kKeyBox, 1024), id_q, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kBM / 16; ++kk) {
+            const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
+            umma_ts(tmem + C::kColDV, tb + kColP + kk * 8,
+                    sdesc_sw128(do_base + kk * 2048, kQBox, 1024), id_kv, acc);
+            umma_ts(tmem + C::kColDK, tb + kColDS + kk * 8,
+                    sdesc_sw128(q_base + kk * 2048, kQBox, 1024), id_kv, acc);
+          }
+          umma_commit(&q_empty[st]);
+          if (n + 2 < n_tiles) {
+            // Buffer b is reused once dQ^T of step n has been read out.
+            if (!mbar_wait(&dq_free[b], (n >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!issue_sdp(n + 2)) { ok = false; break; }
+          }
         }
-        umma_commit(ds_free);
-        umma_commit(dq_full);
-        ++n;
+        umma_commit(acc_done);
+        umma_commit(drain);
+        int dummy = 0;
+        mbar_wait(drain, 0, &dummy);
       }
-      umma_commit(acc_done);
-      umma_commit(drain);
-      int dummy = 0;
-      mbar_wait(drain, 0, &dummy);
+      __syncwarp();
     }
-    __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= 8) {
+    reg_dealloc<kRegsDq>();
     // ------------------------------------------------------------ dQ reduce
     // Each warp owns D/4 columns of dQ (its TMEM lane quarter of dQ^T), stages
     // them as a [64 rows][D/4] fp32 box and adds it to the global accumulator
     // with one tiled TMA reduce-add; no barrier spans more than one warp.
-    const int wq = warp - 4;  // TMEM lane quarter
+    const int wq = warp - 8;  // TMEM lane quarter
     const uint32_t lane_base = uint32_t(wq * 32) << 16;
     // For D = 64 the M = 64 accumulator sits in lanes 0-15 of each quarter.
     const bool valid = (D == 128) || (lane < 16);
-    float* stage0 = sStage + wq * 2 * (C::kStageBytes / 4);
-    int n = 0;
-    for (int qt = c.qt_begin; qt < c.qt_end; ++qt) {
-      if (qtile_class(p, c, qt, qt_bits) == 0) continue;
-      const bool got = mbar_wait(dq_full, n & 1, abort_flag);
-      if (!__all_sync(~0u, got)) break;
+    float* stage = sStage + wq * (C::kStageBytes / 4);
+    for_each_qtile(p, c, [&](int n, int qt, int) -> bool {
+      const int b = n & 1;
+      const bool got = mbar_wait(&dq_full[b], (n >> 1) & 1, abort_flag);
+      if (!__all_sync(~0u, got)) return false;
       tc_fence_after();
       uint32_t r0[32], r1[32];
-      tmem_ld32(tmem + lane_base + C::kColDQ, r0);
-      tmem_ld32(tmem + lane_base + C::kColDQ + 32, r1);
+      tmem_ld32(tmem + lane_base + b * 128 + kColDQ, r0);
+      tmem_ld32(tmem + lane_base + b * 128 + kColDQ + 32, r1);
       tmem_ld_wait(r0);
       tmem_ld_wait(r1);
       tc_fence_before();
-      mbar_arrive(dq_free);
-      float* stage = stage0 + (n & 1) * (C::kStageBytes / 4);
-      // The reduce issued two tiles ago must have finished reading this buffer.
-      if (lane == 0) bulk_wait_group_read1();
+      mbar_arrive(&dq_free[b]);
+      // The previous reduce must have finished reading the stage.
+      if (lane == 0) bulk_wait_group_read0();
       __syncwarp();
       if (valid) {
 #pragma unroll
@@ -352,61 +351,52 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_reduce_add_3d(&tm_dq, stage, col0_dq(D, wq), qt * kBM, c.b * p.N + c.h);
         bulk_commit_group();
       }
-      ++n;
-    }
+      return true;
+    });
     if (lane == 0) bulk_wait_group0();
   } else {
+    reg_alloc<kRegsSoftmax>();
     // ------------------------------------------------------------ softmax
-    const int r = tid;  // key row within the tile, TMEM lane
+    const int g = warp >> 2;             // this warpgroup takes steps n = g mod 2
+    const int wq = warp & 3;             // TMEM lane quarter
+    const int r = wq * 32 + lane;        // key row within the tile
     const int j = c.k0 + r;
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t lane_base = uint32_t(wq * 32) << 16;
     const float sl2 = p.scale_log2;
     const float slope_l2 = p.slopes ? p.slopes[c.h] * kLog2e : 0.f;
     const bool has_alibi = p.slopes != nullptr;
+    const bool causal = p.mask_flags & FA_MASK_CAUSAL;
     const int32_t* ids = (p.mask_flags & FA_MASK_MODALITY) ? p.ids + int64_t(c.b) * p.Sk : nullptr;
-    const int id_j = (ids && j < p.Sk) ? ids[j] : 0;
+    const int id_j = (ids && j < p.Sk) ? (ids[j] & 1) : 0;
     const int64_t row_base = (int64_t(c.b) * p.N + c.h) * p.Sq;
     const uint8_t* mcol = (p.mask_flags & FA_MASK_BOOL)
                               ? p.mask + c.b * p.m_sb + c.h * p.m_sh + j
                               : nullptr;
-    int n = 0;
+    int mine = 0;  // steps of this warpgroup so far
     bool ok = true;
-    for (int qt = c.qt_begin; qt < c.qt_end; ++qt) {
-      const int cls = qtile_class(p, c, qt, qt_bits);
-      if (cls == 0) continue;
+    for_each_qtile(p, c, [&](int n, int qt, int cls) -> bool {
+      if ((n & 1) != g) return true;
+      const int b = n & 1;
       const int q0 = qt * kBM;
-      // Per-row statistics of this query tile (LSE in log2 units), loaded by
-      // each warp into its own buffer.
-      float* st_lse = sStats + warp * 2 * kBM;
-      float* st_dl = st_lse + kBM;
-      __syncwarp();
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int i = q0 + u * 32 + lane;
-        st_lse[u * 32 + lane] = i < p.Sq ? lse[row_base + i] * kLog2e : INFINITY;
-        st_dl[u * 32 + lane] = i < p.Sq ? delta[row_base + i] : 0.f;
+      const uint32_t tb = tmem + lane_base + b * 128;
+      // Row statistics of the 64 queries (LSE in log2 units): lane l holds
+      // queries l and 32 + l; broadcast by shuffles.
+      float lse_lo, lse_hi, dl_lo, dl_hi;
+      {
+        const int i0 = q0 + lane, i1 = q0 + 32 + lane;
+        lse_lo = i0 < p.Sq ? lse[row_base + i0] * kLog2e : INFINITY;
+        lse_hi = i1 < p.Sq ? lse[row_base + i1] * kLog2e : INFINITY;
+        dl_lo = i0 < p.Sq ? delta[row_base + i0] : 0.f;
+        dl_hi = i1 < p.Sq ? delta[row_base + i1] : 0.f;
       }
-      __syncwarp();
-      const bool got_s = mbar_wait(s_full, n & 1, abort_flag);
-      if (!__all_sync(~0u, got_s)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t sr[2][32], dr[2][32];
-      tmem_ld32(tmem + lane_base + kColS, sr[0]);
-      tmem_ld32(tmem + lane_base + kColS + 32, sr[1]);
-      tmem_ld32(tmem + lane_base + kColDP, dr[0]);
-      tmem_ld32(tmem + lane_base + kColDP + 32, dr[1]);
-      tmem_ld_wait(sr[0]);
-      tmem_ld_wait(sr[1]);
-      tmem_ld_wait(dr[0]);
-      tmem_ld_wait(dr[1]);
       // Visibility of the 64 queries of this tile for key j, as bits.
       uint32_t vb[2] = {~0u, ~0u};
       if (cls == 1) {
-        const int lo = (p.mask_flags & FA_MASK_CAUSAL) ? max(0, j - q0) : 0;
+        const int lo = causal ? max(0, j - q0) : 0;
         const int hi = (j < c.nkeys) ? min(kBM, p.Sq - q0) - 1 : -1;
         vb[0] = range_bits(lo, hi, 0);
         vb[1] = range_bits(lo, hi, 1);
-        if (mcol) {
+        if (mcol && j < c.nkeys) {  // column j of the mask exists
 #pragma unroll 1
           for (int w = 0; w < 2; ++w) {
             uint32_t m = 0;
@@ -418,89 +408,113 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ids) {
 #pragma unroll
           for (int w = 0; w < 2; ++w) {
-            uint32_t m = modality_row_bits(p.allow_bits, id_j, qt_bits[qt * 2 + w], false);
+            const int i = q0 + 32 * w + lane;
+            const uint32_t qbits = __ballot_sync(~0u, i < p.Sq && (ids[i < p.Sq ? i : 0] & 1) == 1);
+            uint32_t m = modality_row_bits(p.allow_bits, id_j, qbits, false);
             if (p.allow_bits & 16u) m |= range_bits(j - q0, j - q0, w);
             vb[w] &= m;
           }
         }
       }
-      uint32_t pk[32], dk_[32];
+      const bool got_s = mbar_wait(&s_full[b], mine & 1, abort_flag);
+      if (!__all_sync(~0u, got_s)) { ok = false; return false; }
+      tc_fence_after();
+      // P^T = 2^(s * scale * log2 e + bias - LSE) for the 64 queries.
+      float pf[64];
+      {
+        uint32_t sr[2][32];
+        tmem_ld32(tb + 0, sr[0]);
+        tmem_ld32(tb + 32, sr[1]);
+        tmem_ld_wait(sr[0]);
+        tmem_ld_wait(sr[1]);
+        uint32_t pk[32];
 #pragma unroll
-      for (int e = 0; e < kBM; e += 2) {
-        float pv[2], dsv[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int cc = e + u;
-          const int i = q0 + cc;
-          float t = __uint_as_float(sr[cc >> 5][cc & 31]) * sl2;
-          if (has_alibi) t = fmaf(-slope_l2, float(abs(i - j)), t);
-          const bool vis = (vb[cc >> 5] >> (cc & 31)) & 1u;
-          const float pp = vis ? ex2_approx(t - st_lse[cc]) : 0.f;
-          pv[u] = pp;
-          dsv[u] = pp * (__uint_as_float(dr[cc >> 5][cc & 31]) - st_dl[cc]);
+        for (int e = 0; e < kBM; ++e) {
+          float x = __uint_as_float(sr[e >> 5][e & 31]) * sl2;
+          if (has_alibi) x = fmaf(-slope_l2, float(abs(q0 + e - j)), x);
+          const float l2 = __shfl_sync(~0u, e < 32 ? lse_lo : lse_hi, e & 31);
+          const bool vis = (vb[e >> 5] >> (e & 31)) & 1u;
+          pf[e] = vis ? ex2_approx(x - l2) : 0.f;
         }
-        pk[e >> 1] = pack_bf16x2(pv[0], pv[1]);
-        dk_[e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+#pragma unroll
+        for (int e = 0; e < kBM; e += 2) pk[e >> 1] = pack_bf16x2(pf[e], pf[e + 1]);
+        tmem_st32(tb + kColP, pk);
       }
-      tmem_st32(tmem + lane_base + kColS, pk);
-      tmem_st32(tmem + lane_base + kColDP, dk_);
+      // dS^T = P^T o (dP^T - Delta)
+      uint32_t dsk[32];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t dr[32];
+        tmem_ld32(tb + 64 + hh * 32, dr);
+        tmem_ld_wait(dr);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int cc = hh * 32 + e;
+          const float d0 = __shfl_sync(~0u, hh == 0 ? dl_lo : dl_hi, e);
+          const float d1 = __shfl_sync(~0u, hh == 0 ? dl_lo : dl_hi, e + 1);
+          const float s0 = pf[cc] * (__uint_as_float(dr[e]) - d0);
+          const float s1 = pf[cc + 1] * (__uint_as_float(dr[e + 1]) - d1);
+          dsk[cc >> 1] = pack_bf16x2(s0, s1);
+        }
+      }
+      tmem_st32(tb + kColDS, dsk);
       // dS^T row -> shared memory (128-byte swizzle) for the dQ^T MMA, once
-      // the previous dQ^T MMA has consumed the buffer.
-      if (n > 0) {
-        const bool got_d = mbar_wait(ds_free, (n - 1) & 1, abort_flag);
-        if (!__all_sync(~0u, got_d)) { ok = false; break; }
+      // the dQ^T MMA of this buffer's previous step has consumed it.
+      if (mine > 0) {
+        const bool got_d = mbar_wait(&dq_full[b], (mine - 1) & 1, abort_flag);
+        if (!__all_sync(~0u, got_d)) { ok = false; return false; }
       }
-      uint8_t* row = sDS + r * 128;
+      uint8_t* rowp = sDS + b * 16384 + r * 128;
 #pragma unroll
       for (int ch = 0; ch < 8; ++ch) {
-        *reinterpret_cast<uint4*>(row + ((ch ^ (r & 7)) << 4)) =
-            make_uint4(dk_[4 * ch], dk_[4 * ch + 1], dk_[4 * ch + 2], dk_[4 * ch + 3]);
+        *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) << 4)) =
+            make_uint4(dsk[4 * ch], dsk[4 * ch + 1], dsk[4 * ch + 2], dsk[4 * ch + 3]);
       }
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(p_ready);
-      ++n;
-    }
+      mbar_arrive(&p_ready[b]);
+      ++mine;
+      return true;
+    });
 
     // ---------------------------------------------------------- epilogue
-    const bool have = __all_sync(~0u, ok && n > 0 && mbar_wait(acc_done, 0, abort_flag));
+    // Warpgroup 0 writes dV, warpgroup 1 writes dK (times scale).
+    const int n_tiles = count_qtiles(p, c);
+    const bool have =
+        __all_sync(~0u, ok && n_tiles > 0 && mbar_wait(acc_done, 0, abort_flag));
     if (have) tc_fence_after();
     const bool real = j < p.Sk;
-    __nv_bfloat16* dv_row = dv + c.b * p.k_sb + c.h * p.k_sh + int64_t(j) * p.k_ss;
-    __nv_bfloat16* dk_row = dk + c.b * p.k_sb + c.h * p.k_sh + int64_t(j) * p.k_ss;
+    const int col = g == 0 ? C::kColDV : C::kColDK;
+    const float mul = g == 0 ? 1.f : p.scale;
+    __nv_bfloat16* dst_row =
+        (g == 0 ? dv : dk) + c.b * p.k_sb + c.h * p.k_sh + int64_t(j) * p.k_ss;
 #pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const int col = which == 0 ? kColDV : C::kColDK;
-      const float mul = which == 0 ? 1.f : p.scale;
-      __nv_bfloat16* dst_row = which == 0 ? dv_row : dk_row;
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t a[32];
+      if (have) {
+        tmem_ld32(tmem + lane_base + col + cc * 32, a);
+        tmem_ld_wait(a);
+      }
+      if (real) {
+        uint32_t w[16];
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t a[32];
-        if (have) {
-          tmem_ld32(tmem + lane_base + col + cc * 32, a);
-          tmem_ld_wait(a);
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = have ? __uint_as_float(a[2 * e]) * mul : 0.f;
+          const float x1 = have ? __uint_as_float(a[2 * e + 1]) * mul : 0.f;
+          w[e] = pack_bf16x2(x0, x1);
         }
-        if (real) {
-          uint32_t w[16];
+        uint4* dst = reinterpret_cast<uint4*>(dst_row + cc * 32);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = have ? __uint_as_float(a[2 * e]) * mul : 0.f;
-            const float x1 = have ? __uint_as_float(a[2 * e + 1]) * mul : 0.f;
-            w[e] = pack_bf16x2(x0, x1);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(dst_row + cc * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-        }
+        for (int e = 0; e < 4; ++e)
+          dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
@@ -513,22 +527,21 @@ cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
                          const float* delta, float* dq_acc, void* dk, void* dv,
                          cudaStream_t st) {
   using C = BwdCfg<D>;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   cudaError_t e;
   if ((e = make_operand_map(&tq, q, p, p.Sq, kBM)) != cudaSuccess) return e;
   if ((e = make_operand_map(&tdo, dout, p, p.Sq, kBM)) != cudaSuccess) return e;
   if ((e = make_operand_map(&tk, k, p, p.Sk, kBN)) != cudaSuccess) return e;
   if ((e = make_operand_map(&tv, v, p, p.Sk, kBN)) != cudaSuccess) return e;
-  CUtensorMap tdq;
-  if ((e = make_f32_rows_map(&tdq, dq_acc, p.D, p.Sq, int64_t(p.B) * p.N,
-                             BwdCfg<D>::kDqCols, kBM)) != cudaSuccess)
+  if ((e = make_f32_rows_map(&tdq, dq_acc, p.D, p.Sq, int64_t(p.B) * p.N, C::kDqCols,
+                             kBM)) != cudaSuccess)
     return e;
   e = cudaFuncSetAttribute(bwd_bf16_sm100<D>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((p.Sk + kBN - 1) / kBN, p.N, p.B);
   bwd_bf16_sm100<D><<<grid, kThreads, C::kSmemBytes, st>>>(
-      tq, tk, tv, tdo, tdq, p, lse, delta, dq_acc, static_cast<__nv_bfloat16*>(dk),
+      tq, tk, tv, tdo, tdq, p, lse, delta, static_cast<__nv_bfloat16*>(dk),
       static_cast<__nv_bfloat16*>(dv));
   return cudaGetLastError();
 }
@@ -540,8 +553,6 @@ cudaError_t launch_bwd_bf16_sm100(const Problem& p, const void* q,
                                   const void* dout, const float* lse,
                                   const float* delta, float* dq_acc, void* dk,
                                   void* dv, cudaStream_t st) {
-  if (p.Sq > kMaxQTiles * kBM && (p.mask_flags & FA_MASK_MODALITY))
-    return cudaErrorInvalidValue;
   if (p.D == 64) return launch_bwd_d<64>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
   if (p.D == 128) return launch_bwd_d<128>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
   return cudaErrorInvalidValue;
