@@ -80,6 +80,12 @@ struct FwdCfg {
   // s_full[2], p_full[2], o_final[2], o_empty[2], drain, sched_full[R],
   // sched_empty[R]
   static constexpr int kNumBars = 4 + 2 * kKStages + 2 * kVStages + 8 + 1 + 2 * kSchedRing;
+  // barrier indices
+  static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = bKFull + kKStages;
+  static constexpr int bVFull = bKEmpty + kKStages, bVEmpty = bVFull + kVStages;
+  static constexpr int bSFull = bVEmpty + kVStages, bPFull = bSFull + 2;
+  static constexpr int bOFinal = bPFull + 2, bOEmpty = bOFinal + 2, bDrain = bOEmpty + 2;
+  static constexpr int bSchedFull = bDrain + 1, bSchedEmpty = bSchedFull + kSchedRing;
   static constexpr int kSmemMisc = kSmemBar + kNumBars * 8;  // tmem addr, abort
   static constexpr int kSmemSched = kSmemMisc + 16;           // int[kSchedRing]
   static constexpr int kSmemBytes = kSmemSched + 4 * kSchedRing + 1024;
@@ -216,26 +222,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem + C::kSmemQ;
-  uint8_t* sK = smem + C::kSmemK;
-  uint8_t* sV = smem + C::kSmemV;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
-  uint64_t* q_full = bars;
-  uint64_t* q_empty = q_full + kTiles;
-  uint64_t* k_full = q_empty + kTiles;
-  uint64_t* k_empty = k_full + C::kKStages;
-  uint64_t* v_full = k_empty + C::kKStages;
-  uint64_t* v_empty = v_full + C::kVStages;
-  uint64_t* s_full = v_empty + C::kVStages;
-  uint64_t* p_full = s_full + kTiles;
-  uint64_t* o_final = p_full + kTiles;
-  uint64_t* o_empty = o_final + kTiles;
-  uint64_t* drain = o_empty + kTiles;
-  uint64_t* sched_full = drain + 1;
-  uint64_t* sched_empty = sched_full + kSchedRing;
-  volatile int* sched_ids = reinterpret_cast<volatile int*>(smem + C::kSmemSched);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kSmemMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kSmemMisc + 4);
+  // 32-bit shared-window addresses: only the base lives in a register.
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t sQa = sb + C::kSmemQ, sKa = sb + C::kSmemK, sVa = sb + C::kSmemV;
+  auto BAR = [sb](int i) -> uint32_t { return sb + uint32_t(C::kSmemBar + 8 * i); };
+  const uint32_t tmem_slot = sb + C::kSmemMisc;
+  const uint32_t abort_addr = sb + C::kSmemMisc + 4;
+  const uint32_t never_abort = sb + C::kSmemMisc + 8;  // stays 0: unbounded-abort drains
+  const uint32_t sched_ids = sb + C::kSmemSched;
+  (void)sQa;
 
   const int warp = threadIdx.x >> 5;
   const int tid = threadIdx.x;
@@ -245,37 +240,38 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     for (int t = 0; t < kTiles; ++t) {
-      mbar_init(&q_full[t], 1);
-      mbar_init(&q_empty[t], 1);
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
-      mbar_init(&o_final[t], 1);
-      mbar_init(&o_empty[t], 128);
+      mbar_init(BAR(C::bQFull + t), 1);
+      mbar_init(BAR(C::bQEmpty + t), 1);
+      mbar_init(BAR(C::bSFull + t), 1);
+      mbar_init(BAR(C::bPFull + t), 128);
+      mbar_init(BAR(C::bOFinal + t), 1);
+      mbar_init(BAR(C::bOEmpty + t), 128);
     }
     for (int s = 0; s < C::kKStages; ++s) {
-      mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
+      mbar_init(BAR(C::bKFull + s), 1);
+      mbar_init(BAR(C::bKEmpty + s), 1);
     }
     for (int s = 0; s < C::kVStages; ++s) {
-      mbar_init(&v_full[s], 1);
-      mbar_init(&v_empty[s], 1);
+      mbar_init(BAR(C::bVFull + s), 1);
+      mbar_init(BAR(C::bVEmpty + s), 1);
     }
-    mbar_init(drain, 1);
+    mbar_init(BAR(C::bDrain), 1);
     for (int s = 0; s < kSchedRing; ++s) {
-      mbar_init(&sched_full[s], 1);
-      mbar_init(&sched_empty[s], kSchedConsumers);
+      mbar_init(BAR(C::bSchedFull + s), 1);
+      mbar_init(BAR(C::bSchedEmpty + s), kSchedConsumers);
     }
-    *abort_flag = 0;
+    st_shared_u32(abort_addr, 0u);
+    st_shared_u32(never_abort, 0u);
     fence_barrier_init();
   }
   if (warp == 9) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc_s(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = ld_shared_volatile(tmem_slot);
 
   if (warp >= 8) {
     reg_dealloc<kRegsControl>();
@@ -297,13 +293,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         int w = -1;
         if (lane == 0) {
           if (n >= kSchedRing &&
-              !mbar_wait(&sched_empty[slot], ((n / kSchedRing) - 1) & 1, abort_flag)) {
+              !mbar_wait_s(BAR(C::bSchedEmpty + slot), ((n / kSchedRing) - 1) & 1, abort_addr)) {
             ok = false;
           } else {
             const unsigned int idx = atomicAdd(sched, 1u);
             w = idx < unsigned(n_items) ? int(idx) : -1;
-            sched_ids[slot] = w;
-            mbar_arrive(&sched_full[slot]);
+            st_shared_u32(sched_ids + 4u * slot, uint32_t(w));
+            mbar_arrive(BAR(C::bSchedFull + slot));
           }
         }
         ok = __shfl_sync(~0u, ok, 0);
@@ -318,13 +314,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!has_rows(c, t)) continue;
           if (q_uses[t] > 0) {
             bool got = true;
-            if (lane == 0) got = mbar_wait(&q_empty[t], (q_uses[t] - 1) & 1, abort_flag);
+            if (lane == 0) got = mbar_wait_s(BAR(C::bQEmpty + t), (q_uses[t] - 1) & 1, abort_addr);
             if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
           }
           if (lane == 0 && !(p.debug_flags & 1u)) {  // test hook: never deliver Q
-            mbar_arrive_expect_tx(&q_full[t], C::kTileBytes);
+            mbar_arrive_expect_tx(BAR(C::bQFull + t), C::kTileBytes);
             for (int x = 0; x < C::kBoxes; ++x)
-              tma_load_3d(sQ + t * C::kTileBytes + x * kBoxBytes, &tm_q, &q_full[t],
+              tma_load_3d_s(sQa + t * C::kTileBytes + x * kBoxBytes, &tm_q, BAR(C::bQFull + t),
                           col0 + 64 * x, c.q0[t], z);
           }
           ++q_uses[t];
@@ -336,44 +332,42 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int sk = kidx % C::kKStages, sv = vidx % C::kVStages;
           bool got = true;
           if (lane == 0 && kidx >= C::kKStages)
-            got = mbar_wait(&k_empty[sk], ((kidx / C::kKStages) - 1) & 1, abort_flag);
+            got = mbar_wait_s(BAR(C::bKEmpty + sk), ((kidx / C::kKStages) - 1) & 1, abort_addr);
           if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
           if (lane == 0) {
-            mbar_arrive_expect_tx(&k_full[sk], C::kTileBytes);
+            mbar_arrive_expect_tx(BAR(C::bKFull + sk), C::kTileBytes);
             for (int x = 0; x < C::kBoxes; ++x)
-              tma_load_3d(sK + sk * C::kTileBytes + x * kBoxBytes, &tm_k, &k_full[sk],
+              tma_load_3d_s(sKa + sk * C::kTileBytes + x * kBoxBytes, &tm_k, BAR(C::bKFull + sk),
                           col0 + 64 * x, kt * kBN, z);
           }
           ++kidx;
           if (lane == 0 && vidx >= C::kVStages)
-            got = mbar_wait(&v_empty[sv], ((vidx / C::kVStages) - 1) & 1, abort_flag);
+            got = mbar_wait_s(BAR(C::bVEmpty + sv), ((vidx / C::kVStages) - 1) & 1, abort_addr);
           if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
           if (lane == 0) {
-            mbar_arrive_expect_tx(&v_full[sv], C::kTileBytes);
+            mbar_arrive_expect_tx(BAR(C::bVFull + sv), C::kTileBytes);
             for (int x = 0; x < C::kBoxes; ++x)
-              tma_load_3d(sV + sv * C::kTileBytes + x * kBoxBytes, &tm_v, &v_full[sv],
+              tma_load_3d_s(sVa + sv * C::kTileBytes + x * kBoxBytes, &tm_v, BAR(C::bVFull + sv),
                           col0 + 64 * x, kt * kBN, z);
           }
           ++vidx;
         }
       }
-      if (lane == 0 && *abort_flag) {
+      if (lane == 0 && ld_shared_volatile(abort_addr)) {
         // Let the copies already in flight land before the CTA exits.
-        int dummy = 0;
         for (int u = (kidx > C::kKStages ? kidx - C::kKStages : 0); u < kidx; ++u)
-          mbar_wait(&k_full[u % C::kKStages], (u / C::kKStages) & 1, &dummy);
+          mbar_wait_s(BAR(C::bKFull + u % C::kKStages), (u / C::kKStages) & 1, never_abort);
         for (int u = (vidx > C::kVStages ? vidx - C::kVStages : 0); u < vidx; ++u)
-          mbar_wait(&v_full[u % C::kVStages], (u / C::kVStages) & 1, &dummy);
+          mbar_wait_s(BAR(C::bVFull + u % C::kVStages), (u / C::kVStages) & 1, never_abort);
         if (!(p.debug_flags & 1u))
           for (int t = 0; t < kTiles; ++t)
-            if (q_uses[t] > 0) mbar_wait(&q_full[t], (q_uses[t] - 1) & 1, &dummy);
+            if (q_uses[t] > 0) mbar_wait_s(BAR(C::bQFull + t), (q_uses[t] - 1) & 1, never_abort);
       }
       __syncwarp();
     } else if (warp == 9) {
       // ---------------------------------------------------------- MMA
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      const uint32_t sQa = smem_u32(sQ), sKa = smem_u32(sK), sVa = smem_u32(sV);
       bool ok = true;
       int steps[kTiles] = {0, 0};       // S/P handshakes so far (all items)
       int pend_idx[kTiles] = {-1, -1};  // K/V index whose P V is still to issue
@@ -390,10 +384,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int vi = pend_idx[t];
         const int sv = vi % C::kVStages;
         if (item_pv[t] == 0 && o_uses[t] > 0 &&
-            !mbar_wait(&o_empty[t], (o_uses[t] - 1) & 1, abort_flag))
+            !mbar_wait_s(BAR(C::bOEmpty + t), (o_uses[t] - 1) & 1, abort_addr))
           return false;  // the previous item's O_t has been read out
-        if (!mbar_wait(&p_full[t], (steps[t] - 1) & 1, abort_flag)) return false;
-        if (!mbar_wait(&v_full[sv], (vi / C::kVStages) & 1, abort_flag)) return false;
+        if (!mbar_wait_s(BAR(C::bPFull + t), (steps[t] - 1) & 1, abort_addr)) return false;
+        if (!mbar_wait_s(BAR(C::bVFull + sv), (vi / C::kVStages) & 1, abort_addr)) return false;
         tc_fence_after();
         const uint32_t vbase = sVa + sv * C::kTileBytes;
 #pragma unroll
@@ -403,7 +397,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   (item_pv[t] > 0 || kk > 0) ? 1u : 0u);
         }
         v_users -= 1u << (4 * sv);
-        if (((v_users >> (4 * sv)) & 15u) == 0) umma_commit(&v_empty[sv]);
+        if (((v_users >> (4 * sv)) & 15u) == 0) umma_commit_s(BAR(C::bVEmpty + sv));
         pend_idx[t] = -1;
         ++item_pv[t];
         return true;
@@ -414,9 +408,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int slot = n % kSchedRing;
         int w = -1;
         if (lane == 0) {
-          if (mbar_wait(&sched_full[slot], (n / kSchedRing) & 1, abort_flag)) {
-            w = sched_ids[slot];
-            mbar_arrive(&sched_empty[slot]);
+          if (mbar_wait_s(BAR(C::bSchedFull + slot), (n / kSchedRing) & 1, abort_addr)) {
+            w = int(ld_shared_volatile(sched_ids + 4u * slot));
+            mbar_arrive(BAR(C::bSchedEmpty + slot));
           } else {
             ok = false;
           }
@@ -433,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           item_pv[t] = 0;
           if (!has_rows(c, t)) continue;
           bool got = true;
-          if (lane == 0) got = mbar_wait(&q_full[t], q_uses[t] & 1, abort_flag);
+          if (lane == 0) got = mbar_wait_s(BAR(C::bQFull + t), q_uses[t] & 1, abort_addr);
           if (!__shfl_sync(~0u, got, 0)) ok = false;
           ++q_uses[t];
         }
@@ -446,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (cls0 == 0 && cls1 == 0) continue;
           if (lane == 0) {
             const int sk = idx % C::kKStages;
-            if (!mbar_wait(&k_full[sk], (idx / C::kKStages) & 1, abort_flag)) {
+            if (!mbar_wait_s(BAR(C::bKFull + sk), (idx / C::kKStages) & 1, abort_addr)) {
               ok = false;
             } else {
               tc_fence_after();
@@ -463,12 +457,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                           sdesc_sw128(kbase + off, 16, 1024), idesc_qk,
                           kk > 0 ? 1u : 0u);
                 }
-                umma_commit(&s_full[t]);
+                umma_commit_s(BAR(C::bSFull + t));
                 pend_idx[t] = idx;
                 ++steps[t];
                 v_users += 1u << (4 * (idx % C::kVStages));
               }
-              if (ok) umma_commit(&k_empty[sk]);
+              if (ok) umma_commit_s(BAR(C::bKEmpty + sk));
             }
           }
           ok = __shfl_sync(~0u, ok, 0);
@@ -479,20 +473,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int t = 0; t < kTiles; ++t) {
             if (pend_idx[t] >= 0 && !issue_pv(t)) { ok = false; break; }
             if (item_pv[t] > 0) {
-              umma_commit(&o_final[t]);
+              umma_commit_s(BAR(C::bOFinal + t));
               ++o_uses[t];
             }
             // Q_t may be reloaded once this item's Q K^T are done.
-            if (has_rows(c, t)) umma_commit(&q_empty[t]);
+            if (has_rows(c, t)) umma_commit_s(BAR(C::bQEmpty + t));
           }
         }
         ok = __shfl_sync(~0u, ok, 0);
       }
       if (lane == 0) {
         // Make sure no MMA is in flight when TMEM is released.
-        umma_commit(drain);
-        int dummy = 0;
-        mbar_wait(drain, 0, &dummy);
+        umma_commit_s(BAR(C::bDrain));
+        mbar_wait_s(BAR(C::bDrain), 0, never_abort);
       }
       __syncwarp();
     }
@@ -514,9 +507,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int slot = n % kSchedRing;
       int w = -1;
       if (lane == 0) {
-        if (mbar_wait(&sched_full[slot], (n / kSchedRing) & 1, abort_flag)) {
-          w = sched_ids[slot];
-          mbar_arrive(&sched_empty[slot]);
+        if (mbar_wait_s(BAR(C::bSchedFull + slot), (n / kSchedRing) & 1, abort_addr)) {
+          w = int(ld_shared_volatile(sched_ids + 4u * slot));
+          mbar_arrive(BAR(C::bSchedEmpty + slot));
         } else {
           ok = false;
         }
@@ -545,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int cls = tile_class(p, c, t, kt, kid);
         if (cls == 0) continue;
         // Every wait is agreed warp-wide before the .sync.aligned TMEM ops.
-        const bool got_s = mbar_wait(&s_full[t], steps & 1, abort_flag);
+        const bool got_s = mbar_wait_s(BAR(C::bSFull + t), steps & 1, abort_addr);
         if (!__all_sync(~0u, got_s)) { ok = false; break; }
         tc_fence_after();
         const int k0 = kt * kBN;
@@ -669,7 +662,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         l = l * alpha + (((r[0] + r[1]) + (r[2] + r[3])) + ((r[4] + r[5]) + (r[6] + r[7])));
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&p_full[t]);
+        mbar_arrive(BAR(C::bPFull + t));
         ++steps;
         ++item_steps;
       }
@@ -678,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // -------------------------------------------------------- epilogue
       bool have_o = false;
       if (item_steps > 0) {
-        have_o = __all_sync(~0u, mbar_wait(&o_final[t], o_uses & 1, abort_flag));
+        have_o = __all_sync(~0u, mbar_wait_s(BAR(C::bOFinal + t), o_uses & 1, abort_addr));
         if (!have_o) { ok = false; break; }
         ++o_uses;
         tc_fence_after();
@@ -695,7 +688,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (cc == D / 32 - 1) {
             // O_t has been read: the next item's first P V may overwrite it.
             tc_fence_before();
-            mbar_arrive(&o_empty[t]);
+            mbar_arrive(BAR(C::bOEmpty + t));
           }
         }
         if (row_real) {
@@ -724,7 +717,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (tid == 0 && *abort_flag) atomicOr(p.status, 1u);
+  if (tid == 0 && ld_shared_volatile(abort_addr)) atomicOr(p.status, 1u);
 }
 
 // Work-item counters for the dynamic scheduler, one per launch in flight
