@@ -85,6 +85,8 @@ def lib():
                              vp, vp, vp]
         L.fa_bwd.argtypes = [S, vp, vp, vp, vp, vp, vp, P, M, ctypes.c_float,
                              ctypes.c_float, vp, vp, vp, vp, sz, vp]
+        L.fa_bwd_noalloc.argtypes = [S, vp, vp, vp, vp, vp, vp, P, M, ctypes.c_float,
+                                     ctypes.c_float, vp, vp, vp, vp]
         L.fa_bwd_workspace_size.argtypes = [S]
         L.fa_bwd_workspace_size.restype = sz
         L.fa_mask_tile_map_size.argtypes = [S, M]
@@ -98,7 +100,7 @@ def lib():
         L.fa_status_string.restype = ctypes.c_char_p
         L.fa_version.restype = ctypes.c_char_p
         L.fa_last_cuda_error.restype = ctypes.c_char_p
-        for fn in (L.fa_fwd, L.fa_bwd, L.fa_build_mask_tile_map,
+        for fn in (L.fa_fwd, L.fa_bwd, L.fa_bwd_noalloc, L.fa_build_mask_tile_map,
                    L.fa_build_modality_mask, L.fa_sync_status):
             fn.restype = ctypes.c_int
         _lib = L
@@ -302,6 +304,42 @@ def bwd(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
                           _ptr(workspace), ctypes.c_size_t(workspace.numel()),
                           _stream(query))
     _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20   # FA_NOALLOC_SCRATCH_BYTES of include/fa.h
+
+
+def bwd_noalloc(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
+                pse=None, padding_kv_len=None, atten_mask=None, scale=None, keep_prob=1.0,
+                *, causal=False, modality_ids=None, allow=((1, 1), (0, 1)),
+                allow_diag=False, tile_map=None, dq=None, dk=None, dv=None):
+    """Backward through fa_bwd_noalloc: the library's fixed scratch array
+    replaces the workspace, so the call allocates no scratch (the outputs
+    dq, dk, dv are still the caller's).  Shapes whose workspace would exceed
+    NOALLOC_SCRATCH_BYTES raise FA_ERR_UNSUPPORTED."""
+    if scale is None:
+        raise FaError(FA_ERR_INVALID_ARG, "scale must be given explicitly")
+    shape = make_shape(query, key, head_num, input_layout)
+    for t, n in ((query, "query"), (key, "key"), (value, "value"), (out, "out"),
+                 (dout, "dout")):
+        _check_operand(t, None, n, query)
+    keep = _Keep()
+    m = make_mask(shape, causal=causal, atten_mask=atten_mask,
+                  padding_kv_len=padding_kv_len, modality_ids=modality_ids,
+                  allow=allow, allow_diag=allow_diag, tile_map=tile_map, keep=keep)
+    ps = make_pse(pse, keep)
+    dq = torch.empty_like(query) if dq is None else dq
+    dk = torch.empty_like(key) if dk is None else dk
+    dv = torch.empty_like(value) if dv is None else dv
+    with torch.cuda.device(query.device):
+        st = lib().fa_bwd_noalloc(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
+                                  _ptr(out), _ptr(dout), _ptr(lse),
+                                  None if ps is None else ctypes.byref(ps),
+                                  None if m is None else ctypes.byref(m),
+                                  float(scale), float(keep_prob), _ptr(dq), _ptr(dk),
+                                  _ptr(dv), _stream(query))
+    _check(st, "fa_bwd_noalloc")
     return dq, dk, dv
 
 

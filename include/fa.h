@@ -140,6 +140,32 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
                  float scale, float keep_prob, void* dq, void* dk, void* dv,
                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* Backward without a caller-provided workspace (no counterpart on the source
+ * pages; an addition of this library).  Some callers cannot call cudaMalloc:
+ * code inside a host framework whose memory pool already holds the device
+ * memory, or latency-critical loops that cannot afford the implicit
+ * synchronisation of cudaMalloc / cudaFree.  This entry point allocates
+ * nothing: its scratch (the fp32 dQ accumulator and per-row statistics that
+ * fa_bwd keeps in its workspace) is a fixed device array of
+ * FA_NOALLOC_SCRATCH_BYTES inside the library, reserved on every GPU that
+ * loads the library until the process exits.
+ *   - Arguments, results and errors are those of fa_bwd, except that a
+ *     shape whose fa_bwd_workspace_size() exceeds FA_NOALLOC_SCRATCH_BYTES
+ *     returns FA_ERR_UNSUPPORTED without launching anything.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array: calls that overlap on the GPU (other
+ *     streams, other host threads) race on it and give wrong gradients.
+ *     Calls on one stream, or otherwise ordered, are safe; the array keeps
+ *     the previous call's contents and the backward clears what must start
+ *     at zero. */
+#define FA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void* k,
+                         const void* v, const void* out, const void* dout,
+                         const float* lse, const fa_pse* pse,
+                         const fa_mask* mask, float scale, float keep_prob,
+                         void* dq, void* dk, void* dv, void* stream);
+
 /* Bytes of the tile map for FA_MASK_BOOL with this shape and mask strides:
  * one byte per (b, h or 1 when mask_stride_h == 0, query tile, key tile). */
 size_t fa_mask_tile_map_size(const fa_shape* shape, const fa_mask* mask);
