@@ -68,14 +68,23 @@ struct BwdCfg {
   static constexpr int kSmemQ = kSmemV + kKTile;                 // [stage]
   static constexpr int kSmemDO = kSmemQ + kStages * kQTile;      // [stage]
   static constexpr int kSmemDS = kSmemDO + kStages * kQTile;     // [2] 128 x 64 bf16
-  // dQ staging: per dQ warp one box of 64 rows x (D / 4) fp32 columns
+  // dQ staging: per dQ warp one box of 32 rows x (D / 4) fp32 columns; a
+  // query tile goes out as two such boxes.
   static constexpr int kDqCols = D / 4;
-  static constexpr int kStageBytes = kBM * kDqCols * 4;
+  static constexpr int kDqRows = 32;
+  static constexpr int kStageBytes = kDqRows * kDqCols * 4;
   static constexpr int kSmemStage = kSmemDS + 2 * 128 * 128;
-  static constexpr int kSmemBar = kSmemStage + 4 * kStageBytes;
+  // Per softmax warp: -LSE (log2 units) and -Delta of the current query tile.
+  static constexpr int kSmemStats = kSmemStage + 4 * kStageBytes;
+  static constexpr int kSmemBar = kSmemStats + 8 * 2 * kBM * 4;
   // kv_full, q_full[3], q_empty[3], s_full[2], p_ready[2], dq_full[2],
   // dq_free[2], acc_done, drain
   static constexpr int kNumBars = 1 + 2 * kStages + 8 + 2;
+  // barrier indices
+  static constexpr int bKvFull = 0, bQFull = 1, bQEmpty = 1 + kStages;
+  static constexpr int bSFull = 1 + 2 * kStages, bPReady = bSFull + 2;
+  static constexpr int bDqFull = bPReady + 2, bDqFree = bDqFull + 2;
+  static constexpr int bAccDone = bDqFree + 2, bDrain = bAccDone + 1;
   static constexpr int kSmemMisc = kSmemBar + kNumBars * 8;
   static constexpr int kSmemBytes = kSmemMisc + 16 + 1024;
 };
@@ -148,24 +157,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK = smem + C::kSmemK;
-  uint8_t* sV = smem + C::kSmemV;
-  uint8_t* sQ = smem + C::kSmemQ;
-  uint8_t* sDO = smem + C::kSmemDO;
-  uint8_t* sDS = smem + C::kSmemDS;
+  // 32-bit shared-window addresses: only the base lives in a register.
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t aK = sb + C::kSmemK, aV = sb + C::kSmemV;
+  const uint32_t aQ = sb + C::kSmemQ, aDO = sb + C::kSmemDO, aDS = sb + C::kSmemDS;
+  auto BAR = [sb](int i) -> uint32_t { return sb + uint32_t(C::kSmemBar + 8 * i); };
+  const uint32_t tmem_slot = sb + C::kSmemMisc;
+  const uint32_t abort_addr = sb + C::kSmemMisc + 4;
+  const uint32_t never_abort = sb + C::kSmemMisc + 8;  // stays 0: drains
+  const uint32_t stage_base = sb + C::kSmemStage;
+  uint8_t* sDS = smem + C::kSmemDS;                     // generic, for the dS^T stores
   float* sStage = reinterpret_cast<float*>(smem + C::kSmemStage);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kSmemBar);
-  uint64_t* kv_full = bars;
-  uint64_t* q_full = bars + 1;
-  uint64_t* q_empty = q_full + C::kStages;
-  uint64_t* s_full = q_empty + C::kStages;
-  uint64_t* p_ready = s_full + 2;
-  uint64_t* dq_full = p_ready + 2;
-  uint64_t* dq_free = dq_full + 2;
-  uint64_t* acc_done = dq_free + 2;
-  uint64_t* drain = acc_done + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kSmemMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kSmemMisc + 4);
+  (void)stage_base;
 
   const int warp = threadIdx.x >> 5;
   const int tid = threadIdx.x;
@@ -181,30 +184,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   c.qt_end = (p.Sq + kBM - 1) / kBM;
 
   if (tid == 0) {
-    mbar_init(kv_full, 1);
+    mbar_init(BAR(C::bKvFull), 1);
     for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&q_full[s], 1);
-      mbar_init(&q_empty[s], 1);
+      mbar_init(BAR(C::bQFull + s), 1);
+      mbar_init(BAR(C::bQEmpty + s), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_ready[b], 128);
-      mbar_init(&dq_full[b], 1);
-      mbar_init(&dq_free[b], 128);
+      mbar_init(BAR(C::bSFull + b), 1);
+      mbar_init(BAR(C::bPReady + b), 128);
+      mbar_init(BAR(C::bDqFull + b), 1);
+      mbar_init(BAR(C::bDqFree + b), 128);
     }
-    mbar_init(acc_done, 1);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
+    mbar_init(BAR(C::bAccDone), 1);
+    mbar_init(BAR(C::bDrain), 1);
+    st_shared_u32(abort_addr, 0u);
+    st_shared_u32(never_abort, 0u);
     fence_barrier_init();
   }
   if (warp == 13) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc_s(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
+  const uint32_t tmem = ld_shared_volatile(tmem_slot);
   const bool bsh = p.layout == FA_LAYOUT_BSH;
 
   if (warp >= 12) {
@@ -218,31 +222,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
         tma_prefetch_desc(&tm_do);
-        mbar_arrive_expect_tx(kv_full, 2 * C::kKTile);
+        mbar_arrive_expect_tx(BAR(C::bKvFull), 2 * C::kKTile);
         for (int x = 0; x < C::kBoxes; ++x) {
-          tma_load_3d(sK + x * kKeyBox, &tm_k, kv_full, col0 + 64 * x, c.k0, z);
-          tma_load_3d(sV + x * kKeyBox, &tm_v, kv_full, col0 + 64 * x, c.k0, z);
+          tma_load_3d_s(aK + x * kKeyBox, &tm_k, BAR(C::bKvFull), col0 + 64 * x, c.k0, z);
+          tma_load_3d_s(aV + x * kKeyBox, &tm_v, BAR(C::bKvFull), col0 + 64 * x, c.k0, z);
         }
         int issued = 0;
         for_each_qtile(p, c, [&](int n, int qt, int) -> bool {
           const int st = n % C::kStages, use = n / C::kStages;
-          if (use > 0 && !mbar_wait(&q_empty[st], (use - 1) & 1, abort_flag)) return false;
-          mbar_arrive_expect_tx(&q_full[st], 2 * C::kQTile);
+          if (use > 0 && !mbar_wait_s(BAR(C::bQEmpty + st), (use - 1) & 1, abort_addr)) return false;
+          mbar_arrive_expect_tx(BAR(C::bQFull + st), 2 * C::kQTile);
           for (int x = 0; x < C::kBoxes; ++x) {
-            tma_load_3d(sQ + st * C::kQTile + x * kQBox, &tm_q, &q_full[st],
+            tma_load_3d_s(aQ + st * C::kQTile + x * kQBox, &tm_q, BAR(C::bQFull + st),
                         col0 + 64 * x, qt * kBM, z);
-            tma_load_3d(sDO + st * C::kQTile + x * kQBox, &tm_do, &q_full[st],
+            tma_load_3d_s(aDO + st * C::kQTile + x * kQBox, &tm_do, BAR(C::bQFull + st),
                         col0 + 64 * x, qt * kBM, z);
           }
           issued = n + 1;
           return true;
         });
         // Let every copy this thread issued land before the CTA can exit.
-        int dummy = 0;
-        mbar_wait(kv_full, 0, &dummy);
+        mbar_wait_s(BAR(C::bKvFull), 0, never_abort);
         const int first = issued > C::kStages ? issued - C::kStages : 0;
         for (int u = first; u < issued; ++u)
-          mbar_wait(&q_full[u % C::kStages], (u / C::kStages) & 1, &dummy);
+          mbar_wait_s(BAR(C::bQFull + u % C::kStages), (u / C::kStages) & 1, never_abort);
       }
       __syncwarp();
     } else if (warp == 13) {
@@ -251,14 +254,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr uint32_t id_s = idesc_bf16_f32(128, kBM, 0, 0);  // S^T, dP^T
         constexpr uint32_t id_kv = idesc_bf16_f32(128, D, 0, 1);   // dV, dK
         constexpr uint32_t id_q = idesc_bf16_f32(D, kBM, 1, 1);    // dQ^T
-        const uint32_t aK = smem_u32(sK), aV = smem_u32(sV);
-        const uint32_t aQ = smem_u32(sQ), aDO = smem_u32(sDO), aDS = smem_u32(sDS);
-        const int n_tiles = count_qtiles(p, c);
-        bool ok = mbar_wait(kv_full, 0, abort_flag);
+                const int n_tiles = count_qtiles(p, c);
+        bool ok = mbar_wait_s(BAR(C::bKvFull), 0, abort_addr);
         // S^T = K Q^T and dP^T = V dO^T of step n into buffer n % 2.
         auto issue_sdp = [&](int n) -> bool {
           const int st = n % C::kStages, b = n & 1;
-          if (!mbar_wait(&q_full[st], (n / C::kStages) & 1, abort_flag)) return false;
+          if (!mbar_wait_s(BAR(C::bQFull + st), (n / C::kStages) & 1, abort_addr)) return false;
           tc_fence_after();
           const uint32_t q_base = aQ + st * C::kQTile, do_base = aDO + st * C::kQTile;
           const uint32_t tb = tmem + b * 128;
@@ -271,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_ss(tb + 64, sdesc_sw128(aV + ko, 16, 1024),
                     sdesc_sw128(do_base + qo, 16, 1024), id_s, kk > 0 ? 1u : 0u);
           }
-          umma_commit(&s_full[b]);
+          umma_commit_s(BAR(C::bSFull + b));
           return true;
         };
         if (ok && n_tiles > 0) ok = issue_sdp(0);
@@ -279,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int n = 0; ok && n < n_tiles; ++n) {
           const int st = n % C::kStages, b = n & 1;
           const uint32_t tb = tmem + b * 128;
-          if (!mbar_wait(&p_ready[b], (n >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_s(BAR(C::bPReady + b), (n >> 1) & 1, abort_addr)) { ok = false; break; }
           tc_fence_after();
           // dQ^T = K^T dS^T first, so that its read-out overlaps dV and dK.
 #pragma unroll
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     sdesc_sw128(aDS + b * 16384 + kk * 2048, kKeyBox, 1024), id_q,
                     kk > 0 ? 1u : 0u);
           }
-          umma_commit(&dq_full[b]);
+          umma_commit_s(BAR(C::bDqFull + b));
           // dV += P^T dO ; dK += dS^T Q   (A operands from TMEM)
           const uint32_t q_base = aQ + st * C::kQTile, do_base = aDO + st * C::kQTile;
 #pragma unroll
@@ -299,17 +300,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma_ts(tmem + C::kColDK, tb + kColDS + kk * 8,
                     sdesc_sw128(q_base + kk * 2048, kQBox, 1024), id_kv, acc);
           }
-          umma_commit(&q_empty[st]);
+          umma_commit_s(BAR(C::bQEmpty + st));
           if (n + 2 < n_tiles) {
             // Buffer b is reused once dQ^T of step n has been read out.
-            if (!mbar_wait(&dq_free[b], (n >> 1) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_s(BAR(C::bDqFree + b), (n >> 1) & 1, abort_addr)) { ok = false; break; }
             if (!issue_sdp(n + 2)) { ok = false; break; }
           }
         }
-        umma_commit(acc_done);
-        umma_commit(drain);
-        int dummy = 0;
-        mbar_wait(drain, 0, &dummy);
+        umma_commit_s(BAR(C::bAccDone));
+        umma_commit_s(BAR(C::bDrain));
+        mbar_wait_s(BAR(C::bDrain), 0, never_abort);
       }
       __syncwarp();
     }
@@ -326,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     float* stage = sStage + wq * (C::kStageBytes / 4);
     for_each_qtile(p, c, [&](int n, int qt, int) -> bool {
       const int b = n & 1;
-      const bool got = mbar_wait(&dq_full[b], (n >> 1) & 1, abort_flag);
+      const bool got = mbar_wait_s(BAR(C::bDqFull + b), (n >> 1) & 1, abort_addr);
       if (!__all_sync(~0u, got)) return false;
       tc_fence_after();
       uint32_t r0[32], r1[32];
@@ -335,21 +335,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld_wait(r0);
       tmem_ld_wait(r1);
       tc_fence_before();
-      mbar_arrive(&dq_free[b]);
-      // The previous reduce must have finished reading the stage.
-      if (lane == 0) bulk_wait_group_read0();
-      __syncwarp();
-      if (valid) {
+      mbar_arrive(BAR(C::bDqFree + b));
 #pragma unroll
-        for (int i = 0; i < 32; ++i) stage[i * C::kDqCols + lane] = __uint_as_float(r0[i]);
+      for (int half = 0; half < 2; ++half) {
+        // The previous reduce must have finished reading the stage.
+        if (lane == 0) bulk_wait_group_read0();
+        __syncwarp();
+        if (valid) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) stage[(32 + i) * C::kDqCols + lane] = __uint_as_float(r1[i]);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        tma_reduce_add_3d(&tm_dq, stage, col0_dq(D, wq), qt * kBM, c.b * p.N + c.h);
-        bulk_commit_group();
+          for (int i = 0; i < 32; ++i)
+            stage[i * C::kDqCols + lane] = __uint_as_float(half == 0 ? r0[i] : r1[i]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_reduce_add_3d(&tm_dq, stage, col0_dq(D, wq), qt * kBM + half * C::kDqRows,
+                            c.b * p.N + c.h);
+          bulk_commit_group();
+        }
       }
       return true;
     });
@@ -379,16 +382,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int b = n & 1;
       const int q0 = qt * kBM;
       const uint32_t tb = tmem + lane_base + b * 128;
-      // Row statistics of the 64 queries (LSE in log2 units): lane l holds
-      // queries l and 32 + l; broadcast by shuffles.
-      float lse_lo, lse_hi, dl_lo, dl_hi;
-      {
-        const int i0 = q0 + lane, i1 = q0 + 32 + lane;
-        lse_lo = i0 < p.Sq ? lse[row_base + i0] * kLog2e : INFINITY;
-        lse_hi = i1 < p.Sq ? lse[row_base + i1] * kLog2e : INFINITY;
-        dl_lo = i0 < p.Sq ? delta[row_base + i0] : 0.f;
-        dl_hi = i1 < p.Sq ? delta[row_base + i1] : 0.f;
+      // Row statistics of the 64 queries, negated: -LSE in log2 units and
+      // -Delta, in this warp's own shared buffer (read back as broadcasts).
+      // st[0..63] = -LSE * log2(e), st[64..127] = -Delta (plain shared memory
+      // accesses, so the compiler can schedule the broadcast loads freely).
+      const uint32_t st_w = sb + C::kSmemStats + warp * 2 * kBM * 4;
+      __syncwarp();
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int i = q0 + 32 * u + lane;
+        st_shared_f32(st_w + 4 * (32 * u + lane),
+                      i < p.Sq ? -lse[row_base + i] * kLog2e : -INFINITY);
+        st_shared_f32(st_w + 4 * (kBM + 32 * u + lane), i < p.Sq ? -delta[row_base + i] : 0.f);
       }
+      __syncwarp();
+      const uint32_t st = opaque_u32(st_w);  // reads below follow the writes
       // Visibility of the 64 queries of this tile for key j, as bits.
       uint32_t vb[2] = {~0u, ~0u};
       if (cls == 1) {
@@ -416,10 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      const bool got_s = mbar_wait(&s_full[b], mine & 1, abort_flag);
+      const bool got_s = mbar_wait_s(BAR(C::bSFull + b), mine & 1, abort_addr);
       if (!__all_sync(~0u, got_s)) { ok = false; return false; }
       tc_fence_after();
       // P^T = 2^(s * scale * log2 e + bias - LSE) for the 64 queries.
+      const bool plain = cls == 2 && !has_alibi;
+      const uint64_t sl2x2 = f2_pack(sl2, sl2);
       float pf[64];
       {
         uint32_t sr[2][32];
@@ -427,17 +437,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tb + 32, sr[1]);
         tmem_ld_wait(sr[0]);
         tmem_ld_wait(sr[1]);
+        // x = s * scale * log2(e) - LSE, in place (branch-free)
+#pragma unroll
+        for (int e = 0; e < kBM; e += 2) {
+          const float2 nl = ld_shared_f2(st + 4 * e);
+          float x0, x1;
+          f2_unpack(ffma2(f2_pack(__uint_as_float(sr[e >> 5][e & 31]),
+                                  __uint_as_float(sr[e >> 5][(e & 31) + 1])),
+                          sl2x2, f2_pack(nl.x, nl.y)),
+                    x0, x1);
+          sr[e >> 5][e & 31] = __float_as_uint(x0);
+          sr[e >> 5][(e & 31) + 1] = __float_as_uint(x1);
+        }
+        if (!plain) {
+          // ALiBi bias and the mask, in a loop of their own
+#pragma unroll
+          for (int e = 0; e < kBM; ++e) {
+            float x = __uint_as_float(sr[e >> 5][e & 31]);
+            if (has_alibi) x = fmaf(-slope_l2, float(abs(q0 + e - j)), x);
+            if (!((vb[e >> 5] >> (e & 31)) & 1u)) x = -INFINITY;
+            sr[e >> 5][e & 31] = __float_as_uint(x);
+          }
+        }
         uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < kBM; ++e) {
-          float x = __uint_as_float(sr[e >> 5][e & 31]) * sl2;
-          if (has_alibi) x = fmaf(-slope_l2, float(abs(q0 + e - j)), x);
-          const float l2 = __shfl_sync(~0u, e < 32 ? lse_lo : lse_hi, e & 31);
-          const bool vis = (vb[e >> 5] >> (e & 31)) & 1u;
-          pf[e] = vis ? ex2_approx(x - l2) : 0.f;
+        for (int e = 0; e < kBM; e += 2) {
+          pf[e] = ex2_approx(__uint_as_float(sr[e >> 5][e & 31]));
+          pf[e + 1] = ex2_approx(__uint_as_float(sr[e >> 5][(e & 31) + 1]));
+          pk[e >> 1] = pack_bf16x2(pf[e], pf[e + 1]);
         }
-#pragma unroll
-        for (int e = 0; e < kBM; e += 2) pk[e >> 1] = pack_bf16x2(pf[e], pf[e + 1]);
         tmem_st32(tb + kColP, pk);
       }
       // dS^T = P^T o (dP^T - Delta)
@@ -450,10 +478,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const int cc = hh * 32 + e;
-          const float d0 = __shfl_sync(~0u, hh == 0 ? dl_lo : dl_hi, e);
-          const float d1 = __shfl_sync(~0u, hh == 0 ? dl_lo : dl_hi, e + 1);
-          const float s0 = pf[cc] * (__uint_as_float(dr[e]) - d0);
-          const float s1 = pf[cc + 1] * (__uint_as_float(dr[e + 1]) - d1);
+          const float2 nd = ld_shared_f2(st + 4 * (kBM + cc));
+          const uint64_t t2 = fadd2(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
+                                    f2_pack(nd.x, nd.y));
+          float s0, s1;
+          f2_unpack(fmul2(t2, f2_pack(pf[cc], pf[cc + 1])), s0, s1);
           dsk[cc >> 1] = pack_bf16x2(s0, s1);
         }
       }
@@ -461,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // dS^T row -> shared memory (128-byte swizzle) for the dQ^T MMA, once
       // the dQ^T MMA of this buffer's previous step has consumed it.
       if (mine > 0) {
-        const bool got_d = mbar_wait(&dq_full[b], (mine - 1) & 1, abort_flag);
+        const bool got_d = mbar_wait_s(BAR(C::bDqFull + b), (mine - 1) & 1, abort_addr);
         if (!__all_sync(~0u, got_d)) { ok = false; return false; }
       }
       uint8_t* rowp = sDS + b * 16384 + r * 128;
@@ -473,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       fence_proxy_async_smem();
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_ready[b]);
+      mbar_arrive(BAR(C::bPReady + b));
       ++mine;
       return true;
     });
@@ -482,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Warpgroup 0 writes dV, warpgroup 1 writes dK (times scale).
     const int n_tiles = count_qtiles(p, c);
     const bool have =
-        __all_sync(~0u, ok && n_tiles > 0 && mbar_wait(acc_done, 0, abort_flag));
+        __all_sync(~0u, ok && n_tiles > 0 && mbar_wait_s(BAR(C::bAccDone), 0, abort_addr));
     if (have) tc_fence_after();
     const bool real = j < p.Sk;
     const int col = g == 0 ? C::kColDV : C::kColDK;
@@ -518,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
-  if (tid == 0 && *abort_flag) atomicOr(p.status, 1u);
+  if (tid == 0 && ld_shared_volatile(abort_addr)) atomicOr(p.status, 1u);
 }
 
 template <int D>
@@ -534,7 +563,7 @@ cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
   if ((e = make_operand_map(&tk, k, p, p.Sk, kBN)) != cudaSuccess) return e;
   if ((e = make_operand_map(&tv, v, p, p.Sk, kBN)) != cudaSuccess) return e;
   if ((e = make_f32_rows_map(&tdq, dq_acc, p.D, p.Sq, int64_t(p.B) * p.N, C::kDqCols,
-                             kBM)) != cudaSuccess)
+                             C::kDqRows)) != cudaSuccess)
     return e;
   e = cudaFuncSetAttribute(bwd_bf16_sm100<D>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);

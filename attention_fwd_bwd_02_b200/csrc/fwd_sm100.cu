@@ -65,6 +65,41 @@ constexpr uint32_t kRegsControl = 88;
 static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 
+// 2^x on the FMA pipe, for the share of the exponentials that the MUFU unit
+// (16 results per clock per SM) cannot keep up with.  x = j + f, j = rint(x)
+// by the 1.5 * 2^23 rounding trick, f in [-1/2, 1/2]; 2^f from a cubic with
+// minimax relative error 1.4e-4 (fitted by exp2_fit.py, well below the bf16
+// rounding of P), and j added to the exponent field.  x < -126 gives +0, as
+// the flush-to-zero MUFU path does, so masked (-inf) entries stay exactly 0.
+// Two lanes per call (packed fp32x2 arithmetic).
+__device__ __forceinline__ void exp2_fma_x2(float a0, float a1, float& p0, float& p1) {
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t neg_magic = f2_pack(-12582912.0f, -12582912.0f);
+  const uint64_t minus_one = f2_pack(-1.0f, -1.0f);
+  const uint64_t x2 = f2_pack(a0, a1);
+  const uint64_t y2 = fadd2(x2, magic);         // j in the low mantissa bits
+  const uint64_t j2 = fadd2(y2, neg_magic);     // rint(x), exact
+  const uint64_t f2 = ffma2(j2, minus_one, x2);  // x - j, exact
+  uint64_t q2 = ffma2(f2_pack(0.0551716685295105f, 0.0551716685295105f), f2,
+                      f2_pack(0.2426111251115799f, 0.2426111251115799f));
+  q2 = ffma2(q2, f2, f2_pack(0.6932609677314758f, 0.6932609677314758f));
+  q2 = ffma2(q2, f2, f2_pack(0.9999280571937561f, 0.9999280571937561f));
+  float q0, q1, y0, y1;
+  f2_unpack(q2, q0, q1);
+  f2_unpack(y2, y0, y1);
+  p0 = __int_as_float(__float_as_int(q0) + (__float_as_int(y0) << 23));
+  p1 = __int_as_float(__float_as_int(q1) + (__float_as_int(y1) << 23));
+  p0 = a0 < -126.0f ? 0.0f : p0;
+  p1 = a1 < -126.0f ? 0.0f : p1;
+}
+
+// Pairs (of the 16 in a 32-column chunk) whose exponentials use exp2_fma_x2.
+// Measured on B200 with the current softmax schedule, moving half of them
+// to the FMA pipe (0xAAAA) was slower than the MUFU alone (564 vs 713
+// TFLOP/s, causal S=2048 D=128): the step is issue-bound, not MUFU-bound, so
+// every exponential stays on the MUFU for now.
+constexpr uint32_t kSoftExpPairs = 0x0000u;
+
 template <int D>
 struct FwdCfg {
   static constexpr int kBoxes = D / 64;
@@ -635,8 +670,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t s2 = f2_pack(__uint_as_float(sr[q4][e]), __uint_as_float(sr[q4][e + 1]));
             float a0, a1;
             f2_unpack(plain ? ffma2(s2, sl2x2, neg_m) : fadd2(s2, neg_m), a0, a1);
-            const float p0 = ex2_approx(a0);  // 2^-inf = 0 for masked keys
-            const float p1 = ex2_approx(a1);
+            float p0, p1;
+            if ((kSoftExpPairs >> (e >> 1)) & 1u) {
+              exp2_fma_x2(a0, a1, p0, p1);
+            } else {
+              p0 = ex2_approx(a0);  // 2^-inf = 0 for masked keys
+              p1 = ex2_approx(a1);
+            }
             rs2[(e >> 1) & 3] = fadd2(rs2[(e >> 1) & 3], f2_pack(p0, p1));
             pk[e >> 1] = pack_bf16x2(p0, p1);
           }
