@@ -10,6 +10,7 @@
 #include <stdint.h>
 
 #include "../../include/fa.h"
+#include "../../include/fa_testing.h"
 #include "fa_common.cuh"
 #include "launch.h"
 
@@ -162,13 +163,20 @@ const char* fa_version(void) { return "fa_b200 1.0 sm_100a"; }
 
 const char* fa_last_cuda_error(void) { return cudaGetErrorString(g_last_cuda); }
 
-fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
-                 const void* v, const fa_pse* pse, const fa_mask* mask,
-                 float scale, float keep_prob, void* out, float* lse,
-                 void* stream) {
+}  // extern "C"
+
+namespace {
+
+// fa_fwd with test hooks (debug_flags, see the kernel's Problem).
+fa_status run_fwd(const fa_shape* shape, const void* q, const void* k,
+                  const void* v, const fa_pse* pse, const fa_mask* mask,
+                  float scale, float keep_prob, void* out, float* lse,
+                  void* stream, uint32_t debug_flags) {
   Problem p;
   fa_status st = make_problem(shape, pse, mask, scale, keep_prob, &p);
   if (st != FA_OK) return st;
+  p.debug_flags = debug_flags;
+  if (debug_flags && shape->dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
   if (p.B == 0 || p.N == 0 || p.Sq == 0) return FA_OK;  // nothing to write
   p.status = status_word();
   if (!p.status) return cuda_status(cudaErrorNoDevice);
@@ -186,6 +194,26 @@ fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
   else
     e = fa::launch_fwd_f32(p, q, k, v, out, lse, cs);
   return cuda_status(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
+                 const void* v, const fa_pse* pse, const fa_mask* mask,
+                 float scale, float keep_prob, void* out, float* lse,
+                 void* stream) {
+  return run_fwd(shape, q, k, v, pse, mask, scale, keep_prob, out, lse, stream, 0u);
+}
+
+fa_status fa_testing_fwd_withhold_q(const fa_shape* shape, const void* q,
+                                    const void* k, const void* v,
+                                    const fa_pse* pse, const fa_mask* mask,
+                                    float scale, float keep_prob, void* out,
+                                    float* lse, void* stream) {
+  return run_fwd(shape, q, k, v, pse, mask, scale, keep_prob, out, lse, stream,
+                 fa::kDebugWithholdQ);
 }
 
 size_t fa_bwd_workspace_size(const fa_shape* shape) {

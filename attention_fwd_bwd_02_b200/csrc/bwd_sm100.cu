@@ -257,20 +257,25 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int n_tiles = count_qtiles(p, c);
         bool ok = mbar_wait_s(BAR(C::bKvFull), 0, abort_addr);
         // S^T = K Q^T and dP^T = V dO^T of step n into buffer n % 2.
+        // Operand descriptors as low halves (start address + leading offset);
+        // all operands have an 8-row stride of 1024 B (common high half).
+        constexpr uint32_t kHi = sdesc_hi(1024);
+        const uint32_t k_km = sdesc_lo(aK, 16), v_km = sdesc_lo(aV, 16);
+        const uint32_t q_km = sdesc_lo(aQ, 16), do_km = sdesc_lo(aDO, 16);
+        const uint32_t k_mn = sdesc_lo(aK, kKeyBox), ds_mn = sdesc_lo(aDS, kKeyBox);
+        const uint32_t q_mn = sdesc_lo(aQ, kQBox), do_mn = sdesc_lo(aDO, kQBox);
         auto issue_sdp = [&](int n) -> bool {
           const int st = n % C::kStages, b = n & 1;
           if (!mbar_wait_s(BAR(C::bQFull + st), (n / C::kStages) & 1, abort_addr)) return false;
           tc_fence_after();
-          const uint32_t q_base = aQ + st * C::kQTile, do_base = aDO + st * C::kQTile;
+          const uint32_t so = uint32_t(st) * (C::kQTile >> 4);
           const uint32_t tb = tmem + b * 128;
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t ko = (kk >> 2) * kKeyBox + (kk & 3) * 32;
-            const uint32_t qo = (kk >> 2) * kQBox + (kk & 3) * 32;
-            umma_ss(tb, sdesc_sw128(aK + ko, 16, 1024), sdesc_sw128(q_base + qo, 16, 1024),
-                    id_s, kk > 0 ? 1u : 0u);
-            umma_ss(tb + 64, sdesc_sw128(aV + ko, 16, 1024),
-                    sdesc_sw128(do_base + qo, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+            const uint32_t ko = ((kk >> 2) * kKeyBox + (kk & 3) * 32) >> 4;
+            const uint32_t qo = so + (((kk >> 2) * kQBox + (kk & 3) * 32) >> 4);
+            umma_ss_lh(tb, k_km + ko, kHi, q_km + qo, kHi, id_s, kk > 0 ? 1u : 0u);
+            umma_ss_lh(tb + 64, v_km + ko, kHi, do_km + qo, kHi, id_s, kk > 0 ? 1u : 0u);
           }
           umma_commit_s(BAR(C::bSFull + b));
           return true;
@@ -283,22 +288,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait_s(BAR(C::bPReady + b), (n >> 1) & 1, abort_addr)) { ok = false; break; }
           tc_fence_after();
           // dQ^T = K^T dS^T first, so that its read-out overlaps dV and dK.
+          const uint32_t dso = uint32_t(b) * (16384 >> 4);
 #pragma unroll
-          for (int kk = 0; kk < kBN / 16; ++kk) {
-            umma_ss(tb + kColDQ, sdesc_sw128(aK + kk * 2048, kKeyBox, 1024),
-                    sdesc_sw128(aDS + b * 16384 + kk * 2048, kKeyBox, 1024), id_q,
-                    kk > 0 ? 1u : 0u);
-          }
+          for (int kk = 0; kk < kBN / 16; ++kk)
+            umma_ss_lh(tb + kColDQ, k_mn + kk * (2048 >> 4), kHi, ds_mn + dso + kk * (2048 >> 4),
+                       kHi, id_q, kk > 0 ? 1u : 0u);
           umma_commit_s(BAR(C::bDqFull + b));
           // dV += P^T dO ; dK += dS^T Q   (A operands from TMEM)
-          const uint32_t q_base = aQ + st * C::kQTile, do_base = aDO + st * C::kQTile;
+          const uint32_t so = uint32_t(st) * (C::kQTile >> 4);
+          const uint32_t acc0 = n > 0 ? 1u : 0u;
 #pragma unroll
           for (int kk = 0; kk < kBM / 16; ++kk) {
-            const uint32_t acc = (n > 0 || kk > 0) ? 1u : 0u;
-            umma_ts(tmem + C::kColDV, tb + kColP + kk * 8,
-                    sdesc_sw128(do_base + kk * 2048, kQBox, 1024), id_kv, acc);
-            umma_ts(tmem + C::kColDK, tb + kColDS + kk * 8,
-                    sdesc_sw128(q_base + kk * 2048, kQBox, 1024), id_kv, acc);
+            const uint32_t acc = kk > 0 ? 1u : acc0;
+            umma_ts_lh(tmem + C::kColDV, tb + kColP + kk * 8, do_mn + so + kk * (2048 >> 4), kHi,
+                       id_kv, acc);
+            umma_ts_lh(tmem + C::kColDK, tb + kColDS + kk * 8, q_mn + so + kk * (2048 >> 4), kHi,
+                       id_kv, acc);
           }
           umma_commit_s(BAR(C::bQEmpty + st));
           if (n + 2 < n_tiles) {

@@ -27,9 +27,14 @@ struct Problem {
   const int32_t* ids;       // modality ids [B][Sk]
   uint32_t allow_bits;      // bit (2*id_q + id_k): allowed; bit 4: diagonal
   const float* slopes;      // ALiBi slopes [N] or null
-  uint32_t debug_flags;     // test hooks (include/fa_testing.h)
+  uint32_t debug_flags;     // test hooks, 0 in production (kDebug* below)
   unsigned int* status;     // device status word (bit 0: a wait timed out)
 };
+
+// Test hook of fa_testing_fwd_withhold_q: the forward's TMA producer never
+// delivers the Q tiles, so every bounded wait on them expires.
+constexpr uint32_t kDebugWithholdQ = 1u;
+
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;

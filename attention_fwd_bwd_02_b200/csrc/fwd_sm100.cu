@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) got = mbar_wait_s(BAR(C::bQEmpty + t), (q_uses[t] - 1) & 1, abort_addr);
             if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
           }
-          if (lane == 0 && !(p.debug_flags & 1u)) {  // test hook: never deliver Q
+          if (lane == 0 && !(p.debug_flags & kDebugWithholdQ)) {
             mbar_arrive_expect_tx(BAR(C::bQFull + t), C::kTileBytes);
             for (int x = 0; x < C::kBoxes; ++x)
               tma_load_3d_s(sQa + t * C::kTileBytes + x * kBoxBytes, &tm_q, BAR(C::bQFull + t),
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait_s(BAR(C::bKFull + u % C::kKStages), (u / C::kKStages) & 1, never_abort);
         for (int u = (vidx > C::kVStages ? vidx - C::kVStages : 0); u < vidx; ++u)
           mbar_wait_s(BAR(C::bVFull + u % C::kVStages), (u / C::kVStages) & 1, never_abort);
-        if (!(p.debug_flags & 1u))
+        if (!(p.debug_flags & kDebugWithholdQ))
           for (int t = 0; t < kTiles; ++t)
             if (q_uses[t] > 0) mbar_wait_s(BAR(C::bQFull + t), (q_uses[t] - 1) & 1, never_abort);
       }
@@ -403,6 +403,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ---------------------------------------------------------- MMA
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBN, 0, 0);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      // Operand descriptors as low halves (start address + leading offset);
+      // every operand here has an 8-row stride of 1024 B (common high half).
+      // Q and K are K-major (64-column boxes); V is N-major with a box of
+      // 64 columns per leading step.
+      constexpr uint32_t kDescHi = sdesc_hi(1024);
+      const uint32_t q_lo = sdesc_lo(sQa, 16), k_lo = sdesc_lo(sKa, 16);
+      const uint32_t v_lo = sdesc_lo(sVa, kBoxBytes);
       bool ok = true;
       int steps[kTiles] = {0, 0};       // S/P handshakes so far (all items)
       int pend_idx[kTiles] = {-1, -1};  // K/V index whose P V is still to issue
@@ -424,13 +431,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait_s(BAR(C::bPFull + t), (steps[t] - 1) & 1, abort_addr)) return false;
         if (!mbar_wait_s(BAR(C::bVFull + sv), (vi / C::kVStages) & 1, abort_addr)) return false;
         tc_fence_after();
-        const uint32_t vbase = sVa + sv * C::kTileBytes;
+        const uint32_t vd = v_lo + uint32_t(sv) * (C::kTileBytes >> 4);
+        const uint32_t acc0 = item_pv[t] > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bdesc = sdesc_sw128(vbase + kk * 2048, kBoxBytes, 1024);
-          umma_ts(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8, bdesc, idesc_pv,
-                  (item_pv[t] > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ts_lh(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8, vd + kk * (2048 >> 4),
+                     kDescHi, idesc_pv, kk > 0 ? 1u : acc0);
         v_users -= 1u << (4 * sv);
         if (((v_users >> (4 * sv)) & 15u) == 0) umma_commit_s(BAR(C::bVEmpty + sv));
         pend_idx[t] = -1;
@@ -479,18 +485,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               ok = false;
             } else {
               tc_fence_after();
-              const uint32_t kbase = sKa + sk * C::kTileBytes;
+              const uint32_t kd = k_lo + uint32_t(sk) * (C::kTileBytes >> 4);
 #pragma unroll
               for (int t = 0; t < kTiles; ++t) {
                 if (pend_idx[t] >= 0 && !issue_pv(t)) { ok = false; break; }
                 if ((t == 0 ? cls0 : cls1) == 0) continue;
-                const uint32_t qbase = sQa + t * C::kTileBytes;
+                const uint32_t qd = q_lo + t * (C::kTileBytes >> 4);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                  const uint32_t off = (kk >> 2) * kBoxBytes + (kk & 3) * 32;
-                  umma_ss(tmem + t * 128, sdesc_sw128(qbase + off, 16, 1024),
-                          sdesc_sw128(kbase + off, 16, 1024), idesc_qk,
-                          kk > 0 ? 1u : 0u);
+                  const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+                  umma_ss_lh(tmem + t * 128, qd + off, kDescHi, kd + off, kDescHi, idesc_qk,
+                             kk > 0 ? 1u : 0u);
                 }
                 umma_commit_s(BAR(C::bSFull + t));
                 pend_idx[t] = idx;
@@ -637,15 +642,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 128; ++e)
             if (!((vb[e >> 5] >> (e & 31)) & 1u)) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
         }
-        // Row max with 8 independent chains.
+        // Row max: three-input max, 8 independent chains.
         float mx8[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) mx8[u] = __uint_as_float(sr[0][u]);
+        for (int u = 0; u < 8; ++u)
+          mx8[u] = fmaxf(__uint_as_float(sr[0][u]), __uint_as_float(sr[0][u + 8]));
 #pragma unroll
-        for (int e = 8; e < 128; ++e)
-          mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sr[e >> 5][e & 31]));
-        float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                         fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int e = 16; e < 128; e += 16) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            mx8[u] = fmax3(mx8[u], __uint_as_float(sr[(e + u) >> 5][(e + u) & 31]),
+                           __uint_as_float(sr[(e + 8 + u) >> 5][(e + 8 + u) & 31]));
+        }
+        float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                         fmaxf(mx8[6], mx8[7]));
         if (plain) mx *= sl2;  // -inf stays -inf (sl2 > 0)
         // Move the reference max only when it grew by more than 2^8: O and l
         // are then rescaled by alpha (exact after the final division).

@@ -22,6 +22,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "fa.h")
+TESTING_HEADER = os.path.join(os.path.dirname(_HERE), "include", "fa_testing.h")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 FA_LAYOUT_BNSD, FA_LAYOUT_BSH = 0, 1
@@ -87,6 +88,7 @@ def lib():
                              ctypes.c_float, vp, vp, vp, vp, sz, vp]
         L.fa_bwd_noalloc.argtypes = [S, vp, vp, vp, vp, vp, vp, P, M, ctypes.c_float,
                                      ctypes.c_float, vp, vp, vp, vp]
+        L.fa_testing_fwd_withhold_q.argtypes = L.fa_fwd.argtypes
         L.fa_bwd_workspace_size.argtypes = [S]
         L.fa_bwd_workspace_size.restype = sz
         L.fa_mask_tile_map_size.argtypes = [S, M]
@@ -100,7 +102,8 @@ def lib():
         L.fa_status_string.restype = ctypes.c_char_p
         L.fa_version.restype = ctypes.c_char_p
         L.fa_last_cuda_error.restype = ctypes.c_char_p
-        for fn in (L.fa_fwd, L.fa_bwd, L.fa_bwd_noalloc, L.fa_build_mask_tile_map,
+        for fn in (L.fa_fwd, L.fa_testing_fwd_withhold_q, L.fa_bwd, L.fa_bwd_noalloc,
+                   L.fa_build_mask_tile_map,
                    L.fa_build_modality_mask, L.fa_sync_status):
             fn.restype = ctypes.c_int
         _lib = L
@@ -108,7 +111,7 @@ def lib():
 
 
 def declared_functions(header: str = HEADER):
-    """Names of the functions include/fa.h declares."""
+    """Names of the functions a header of include/ declares."""
     txt = open(header).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
     return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", txt)))
@@ -235,7 +238,8 @@ def make_pse(slopes: Optional[torch.Tensor], keep: _Keep) -> Optional[FaPse]:
 def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
         padding_kv_len=None, atten_mask=None, scale=None, keep_prob=1.0, *,
         causal=False, modality_ids=None, allow=((1, 1), (0, 1)), allow_diag=False,
-        tile_map=None, out=None, lse=None) -> Tuple[torch.Tensor, torch.Tensor]:
+        tile_map=None, out=None, lse=None,
+        _withhold_q=False) -> Tuple[torch.Tensor, torch.Tensor]:
     """Fused attention forward.  Returns (out, lse).
 
     pse: ALiBi slope vector [N] (fp32) or None.  atten_mask: bool/uint8
@@ -259,14 +263,24 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
     if lse is None:
         lse = torch.empty((shape.B, shape.N, shape.Sq), dtype=torch.float32,
                           device=query.device)
+    entry = lib().fa_testing_fwd_withhold_q if _withhold_q else lib().fa_fwd
     with torch.cuda.device(query.device):
-        st = lib().fa_fwd(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
-                          None if ps is None else ctypes.byref(ps),
-                          None if m is None else ctypes.byref(m),
-                          float(scale), float(keep_prob), _ptr(out), _ptr(lse),
-                          _stream(query))
+        st = entry(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
+                   None if ps is None else ctypes.byref(ps),
+                   None if m is None else ctypes.byref(m),
+                   float(scale), float(keep_prob), _ptr(out), _ptr(lse),
+                   _stream(query))
     _check(st, "fa_fwd")
     return out, lse
+
+
+def testing_fwd_withhold_q(query, key, value, head_num=None, input_layout="BNSD",
+                           scale=None, **kw):
+    """Test only (include/fa_testing.h): the forward with its query tiles
+    withheld, so that its bounded waits expire.  The next sync_status()
+    raises FaError(FA_ERR_TIMEOUT)."""
+    return fwd(query, key, value, head_num, input_layout, scale=scale,
+               _withhold_q=True, **kw)
 
 
 def bwd_workspace_size(shape: FaShape) -> int:

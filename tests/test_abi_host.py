@@ -22,6 +22,19 @@ def test_exports_every_declared_function(L):
     assert "fa_fwd" in names and "fa_bwd" in names
     for n in names:
         assert hasattr(L, n), f"{n} declared in fa.h but not exported"
+    testing = fa.declared_functions(fa.TESTING_HEADER)
+    assert testing == ["fa_testing_fwd_withhold_q"]
+    for n in testing:
+        assert hasattr(L, n), f"{n} declared in fa_testing.h but not exported"
+
+
+def test_testing_entry_validates_like_fwd(L):
+    # Same validation as fa_fwd, before any device work; fp32 has no hook.
+    args = lambda shape: (ctypes.byref(shape), FAKE, FAKE, FAKE, None, None,
+                          0.125, 1.0, FAKE, FAKE, None)
+    assert L.fa_testing_fwd_withhold_q(*args(_shape(D=96))) == fa.FA_ERR_UNSUPPORTED
+    assert L.fa_testing_fwd_withhold_q(*args(_shape(B=-1))) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_testing_fwd_withhold_q(*args(_shape(dtype=fa.FA_F32))) == fa.FA_ERR_UNSUPPORTED
 
 
 def test_status_strings_and_version(L):
