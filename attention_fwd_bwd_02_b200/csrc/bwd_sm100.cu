@@ -573,6 +573,18 @@ cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
   e = cudaFuncSetAttribute(bwd_bf16_sm100<D>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  // The register split (setmaxnreg) draws on the launch allocation of
+  // 65536 / kThreads registers per thread; a build with fewer would leave
+  // the increase waiting.
+  static int regs_ok[2] = {0, 0};
+  if (!regs_ok[D == 128]) {
+    cudaFuncAttributes fa_attr;
+    if ((e = cudaFuncGetAttributes(&fa_attr, bwd_bf16_sm100<D>)) != cudaSuccess) return e;
+    if (fa_attr.numRegs * kThreads < 2 * 128 * int(kRegsSoftmax) + 128 * int(kRegsDq) +
+                                         128 * int(kRegsControl))
+      return cudaErrorInvalidConfiguration;
+    regs_ok[D == 128] = 1;
+  }
   dim3 grid((p.Sk + kBN - 1) / kBN, p.N, p.B);
   bwd_bf16_sm100<D><<<grid, kThreads, C::kSmemBytes, st>>>(
       tq, tk, tv, tdo, tdq, p, lse, delta, static_cast<__nv_bfloat16*>(dk),

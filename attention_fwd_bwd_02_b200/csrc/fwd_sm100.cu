@@ -818,6 +818,15 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmemBytes);
   if (e != cudaSuccess) return e;
+  // The register split (setmaxnreg) draws on the launch allocation; a build
+  // with fewer registers per thread would leave the increase waiting.
+  static int regs_ok[2] = {0, 0};
+  if (!regs_ok[D == 128]) {
+    cudaFuncAttributes fa_attr;
+    if ((e = cudaFuncGetAttributes(&fa_attr, fwd_bf16_sm100<D>)) != cudaSuccess) return e;
+    if (fa_attr.numRegs < int(kRegsLaunch)) return cudaErrorInvalidConfiguration;
+    regs_ok[D == 128] = 1;
+  }
   const int q_blocks = (p.Sq + kRows - 1) / kRows;
   const int64_t items = int64_t(q_blocks) * p.B * p.N;
   if (items > 0x7fffffff) return cudaErrorInvalidValue;
