@@ -114,6 +114,128 @@ __global__ void bwd_post_kernel(Problem p, const float* __restrict__ dq_acc,
   }
 }
 
+// Vectorised forms of bwd_pre / bwd_post for rows of 16-byte chunks: each
+// lane owns one 16-byte chunk (kVE elements) of a row and LPR lanes cover a
+// row, so a warp moves 32 / LPR rows per pass; every lane keeps two passes
+// of loads in flight.  Row r of the [B][N][Sq] enumeration lives at
+// b * q_sb + h * q_sh + i * q_ss in either layout.
+template <typename T>
+struct Vec16 {
+  static constexpr int kVE = 16 / int(sizeof(T));
+};
+
+__device__ __forceinline__ int64_t row_offset(const Problem& p, int64_t r) {
+  const int i = int(r % p.Sq);
+  const int64_t bh = r / p.Sq;
+  const int h = int(bh % p.N), b = int(bh / p.N);
+  return b * p.q_sb + h * p.q_sh + int64_t(i) * p.q_ss;
+}
+
+// 16 bytes of T as floats (kVE of them).
+__device__ __forceinline__ void load16(const float* p, float (&v)[4]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+}
+__device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    v[2 * k] = __uint_as_float(w[k] << 16);
+    v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+  }
+}
+__device__ __forceinline__ void store16(float* p, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+__device__ __forceinline__ void store16(__nv_bfloat16* p, const float (&v)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+    w[k] = *reinterpret_cast<const uint32_t*>(&h2);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <typename T, int LPR>
+__global__ void bwd_pre_vec_kernel(Problem p, const T* __restrict__ out,
+                                   const T* __restrict__ dout,
+                                   float* __restrict__ delta,
+                                   float* __restrict__ dq_acc) {
+  constexpr int kVE = Vec16<T>::kVE;
+  constexpr int kRPW = 32 / LPR;  // rows per warp per pass
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, li = lane % LPR;
+  const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  const int64_t warp = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int64_t base = warp * 2 * kRPW; base < rows; base += nwarps * 2 * kRPW) {
+    float a[2][kVE] = {}, o[2][kVE] = {};
+    int64_t r[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      r[u] = base + u * kRPW + sub;
+      if (r[u] < rows) {
+        const int64_t off = row_offset(p, r[u]) + li * kVE;
+        load16(dout + off, a[u]);
+        load16(out + off, o[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < kVE; ++e) acc = fmaf(a[u][e], o[u][e], acc);
+#pragma unroll
+      for (int m = LPR / 2; m; m >>= 1) acc += __shfl_xor_sync(~0u, acc, m);
+      if (r[u] < rows) {
+        // this lane's kVE fp32 of the accumulator row: kVE * 4 bytes
+        float4* z = reinterpret_cast<float4*>(dq_acc + r[u] * p.D + li * kVE);
+#pragma unroll
+        for (int k = 0; k < kVE / 4; ++k) z[k] = zero;
+        if (li == 0) delta[r[u]] = acc;
+      }
+    }
+  }
+}
+
+template <typename T, int LPR>
+__global__ void bwd_post_vec_kernel(Problem p, const float* __restrict__ dq_acc,
+                                    T* __restrict__ dq) {
+  constexpr int kVE = Vec16<T>::kVE;
+  constexpr int kRPW = 32 / LPR;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, li = lane % LPR;
+  const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  const int64_t warp = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int64_t nwarps = int64_t(gridDim.x) * (blockDim.x >> 5);
+  for (int64_t base = warp * 2 * kRPW; base < rows; base += nwarps * 2 * kRPW) {
+    float v[2][kVE];
+    int64_t r[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      r[u] = base + u * kRPW + sub;
+      if (r[u] < rows) {
+        const float* src = dq_acc + r[u] * p.D + li * kVE;
+#pragma unroll
+        for (int k = 0; k < kVE / 4; ++k) {
+          const float4 x = reinterpret_cast<const float4*>(src)[k];
+          v[u][4 * k] = x.x; v[u][4 * k + 1] = x.y; v[u][4 * k + 2] = x.z; v[u][4 * k + 3] = x.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      if (r[u] >= rows) continue;
+#pragma unroll
+      for (int e = 0; e < kVE; ++e) v[u][e] *= p.scale;
+      store16(dq + row_offset(p, r[u]) + li * kVE, v[u]);
+    }
+  }
+}
+
 // One CTA per tile: 256 threads scan the 128 x 128 bytes of the mask tile.
 __global__ void tile_map_kernel(Problem p, uint8_t* __restrict__ tile_map) {
   const int nqt = (p.Sq + FA_TILE_M - 1) / FA_TILE_M;
@@ -189,10 +311,47 @@ cudaError_t launch_fill_empty_rows(const Problem& p, bool is_bf16, void* out,
   return cudaGetLastError();
 }
 
+// Lanes per row of the vectorised kernels (16-byte chunks), 0 if the row
+// does not split into a power-of-two number of chunks of at most 32.
+int lanes_per_row(const Problem& p, bool is_bf16) {
+  const int ve = is_bf16 ? 8 : 4;
+  if (p.D % ve != 0) return 0;
+  const int lpr = p.D / ve;
+  return (lpr == 8 || lpr == 16 || lpr == 32) ? lpr : 0;
+}
+
+template <typename T>
+cudaError_t pre_vec(const Problem& p, int lpr, int g, const void* out, const void* dout,
+                    float* delta, float* dq_acc, cudaStream_t st) {
+  const T* o = static_cast<const T*>(out);
+  const T* d = static_cast<const T*>(dout);
+  if (lpr == 8) bwd_pre_vec_kernel<T, 8><<<g, 256, 0, st>>>(p, o, d, delta, dq_acc);
+  else if (lpr == 16) bwd_pre_vec_kernel<T, 16><<<g, 256, 0, st>>>(p, o, d, delta, dq_acc);
+  else bwd_pre_vec_kernel<T, 32><<<g, 256, 0, st>>>(p, o, d, delta, dq_acc);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t post_vec(const Problem& p, int lpr, int g, const float* dq_acc, void* dq,
+                     cudaStream_t st) {
+  T* q = static_cast<T*>(dq);
+  if (lpr == 8) bwd_post_vec_kernel<T, 8><<<g, 256, 0, st>>>(p, dq_acc, q);
+  else if (lpr == 16) bwd_post_vec_kernel<T, 16><<<g, 256, 0, st>>>(p, dq_acc, q);
+  else bwd_post_vec_kernel<T, 32><<<g, 256, 0, st>>>(p, dq_acc, q);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bwd_pre(const Problem& p, bool is_bf16, const void* out,
                            const void* dout, float* delta, float* dq_acc,
                            cudaStream_t st) {
   const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  const int lpr = lanes_per_row(p, is_bf16);
+  if (lpr) {
+    // 8 warps per block, each covering 2 passes of 32 / lpr rows.
+    const int g = grid_for(rows, 8 * 2 * (32 / lpr));
+    return is_bf16 ? pre_vec<__nv_bfloat16>(p, lpr, g, out, dout, delta, dq_acc, st)
+                   : pre_vec<float>(p, lpr, g, out, dout, delta, dq_acc, st);
+  }
   const int g = grid_for(rows, 8);
   if (is_bf16)
     bwd_pre_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
@@ -208,6 +367,12 @@ cudaError_t launch_bwd_pre(const Problem& p, bool is_bf16, const void* out,
 cudaError_t launch_bwd_post(const Problem& p, bool is_bf16,
                             const float* dq_acc, void* dq, cudaStream_t st) {
   const int64_t rows = int64_t(p.B) * p.N * p.Sq;
+  const int lpr = lanes_per_row(p, is_bf16);
+  if (lpr) {
+    const int g = grid_for(rows, 8 * 2 * (32 / lpr));
+    return is_bf16 ? post_vec<__nv_bfloat16>(p, lpr, g, dq_acc, dq, st)
+                   : post_vec<float>(p, lpr, g, dq_acc, dq, st);
+  }
   const int g = grid_for(rows, 8);
   if (is_bf16)
     bwd_post_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
