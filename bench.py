@@ -165,7 +165,9 @@ class ClockSampler:
                 "source": "nvml, 20 ms period, warm-up and timed region"}
 
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend=None):
+    """Joins the process group of a torchrun launch (one rank per GPU).  The
+    backend is NCCL on GPUs; gloo serves the CPU tests of this plumbing."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -173,18 +175,30 @@ def dist_setup(n_gpus):
         import torch.distributed as dist
         from datetime import timedelta
         import torch
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        backend = backend or "nccl"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timedelta(seconds=120))
     return rank, world, local
 
 
+def _collective_device():
+    import torch
+    import torch.distributed as dist
+    return torch.device("cuda", torch.cuda.current_device()) \
+        if dist.get_backend() == "nccl" else torch.device("cpu")
+
+
 def max_over_ranks(x, world):
+    """The largest of every rank's x (each rank's own device timing)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_collective_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -193,6 +207,12 @@ def barrier(world):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
+
+
+def whole_job_value(step_flops_per_rank, world, ms_per_step):
+    """Whole-job throughput (TFLOP/s): every rank runs the same workload
+    (weak scaling), the step time is the slowest rank's."""
+    return step_flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
 
 
 def run_ours(args):
@@ -294,7 +314,7 @@ def run_ours(args):
         return
     pk, pk_kind = peaks()
     ms_step = total_ms / args.steps
-    value = STEP_FLOPS * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_value(STEP_FLOPS, world, ms_step)
     fwd_tf = FWD_FLOPS / (fwd_ms * 1e-3) / 1e12
     bwd_tf = BWD_FLOPS / (bwd_ms * 1e-3) / 1e12
     peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
@@ -342,7 +362,7 @@ def run_ours(args):
                          bwd_ms if dominant == "bwd" else fwd_ms),
         "roofline_fwd": roof("fwd", fwd_tf, fwd_ms),
         "cpu_baseline": cpu,
-        "e2e": {"value": round(STEP_FLOPS * world / (e2e_ms * 1e-3) / 1e12, 2),
+        "e2e": {"value": round(whole_job_value(STEP_FLOPS, world, e2e_ms), 2),
                 "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(e2e_ms, 4)},
         "gpu_launches": 4 * args.steps,
