@@ -135,8 +135,18 @@ struct Item {
   uint32_t q_ids[kTiles];          // modality: bit a set if some row has id a
 };
 
+// Per-tile fields of an item read with selects rather than an indexed
+// load: with a run-time t (the softmax warpgroup's tile) an indexed access
+// would place the item in local memory.
+__device__ __forceinline__ int item_q0(const Item& c, int t) { return t ? c.q0[1] : c.q0[0]; }
+__device__ __forceinline__ int item_q_last(const Item& c, int t) {
+  return t ? c.q_last[1] : c.q_last[0];
+}
+__device__ __forceinline__ uint32_t item_q_ids(const Item& c, int t) {
+  return t ? c.q_ids[1] : c.q_ids[0];
+}
 __device__ __forceinline__ bool has_rows(const Item& c, int t) {
-  return c.q_last[t] >= c.q0[t];
+  return item_q_last(c, t) >= item_q0(c, t);
 }
 
 // Work item number idx of the claim order.  Heads are taken in groups of
@@ -205,7 +215,7 @@ __device__ __forceinline__ uint32_t key_tile_ids(const Problem& p, const Item& c
 // 0 = nothing visible, 1 = partly visible (mask per element), 2 = all visible.
 __device__ __forceinline__ int tile_class(const Problem& p, const Item& c, int t,
                                           int kt, uint32_t k_ids) {
-  const int q0 = c.q0[t], q_last = c.q_last[t];
+  const int q0 = item_q0(c, t), q_last = item_q_last(c, t);
   if (q_last < q0) return 0;
   const int k0 = kt * kBN;
   if (k0 >= c.nkeys) return 0;
@@ -233,7 +243,7 @@ __device__ __forceinline__ int tile_class(const Problem& p, const Item& c, int t
     for (int a = 0; a < 2; ++a)
 #pragma unroll
       for (int e = 0; e < 2; ++e)
-        if (((c.q_ids[t] >> a) & 1u) && ((k_ids >> e) & 1u)) {
+        if (((item_q_ids(c, t) >> a) & 1u) && ((k_ids >> e) & 1u)) {
           const bool ok = (p.allow_bits >> (a * 2 + e)) & 1u;
           any |= ok;
           all &= ok;
@@ -560,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Item c = make_item(p, w, q_blocks, group, causal);
       item_query_ids(p, c);
       if (!has_rows(c, t)) continue;
-      const int i = c.q0[t] + row;  // query index
+      const int i = item_q0(c, t) + row;  // query index
       const bool row_real = i < p.Sq;
       const float slope_l2 = has_alibi ? p.slopes[c.h] * kLog2e : 0.f;
       const int32_t* ids =

@@ -81,9 +81,34 @@ def committed_traffic():
     return d.get("kernels", {})
 
 
+_SAMPLER = r"""
+import sys, time
+import pynvml as nv
+nv.nvmlInit()
+bus = sys.argv[1]
+try:
+    h = nv.nvmlDeviceGetHandleByPciBusId(bus)
+except Exception:
+    h = nv.nvmlDeviceGetHandleByIndex(int(sys.argv[2]))
+mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+period = float(sys.argv[3])
+out = sys.stdout
+while True:
+    try:
+        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+    except Exception:
+        pw = -1.0
+    out.write("%d %d %.1f %d\n" % (nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), mx, pw,
+                                    nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+    out.flush()
+    time.sleep(period)
+"""
+
+
 class ClockSampler:
-    """Samples SM clocks and clock-event (throttle) reasons through NVML on a
-    background thread every 20 ms while the GPU works."""
+    """Samples SM clocks, power and clock-event (throttle) reasons through
+    NVML every 2 ms while the GPU works.  The sampler is a separate process,
+    so the benchmark's own Python thread cannot starve it."""
 
     REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
                ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
@@ -91,70 +116,74 @@ class ClockSampler:
                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
                ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, cuda_index, period_s=0.02):
+    def __init__(self, cuda_index, period_s=0.002):
         self.cuda_index = cuda_index
         self.period = period_s
         self.samples = []          # (sm_mhz, max_mhz, power_w, reason_bits)
         self.error = None
-        self._stop = threading.Event()
-        self._thread = None
+        self.proc = None
+        self._reader = None
+        self._on = False
 
-    def _handle(self, nv):
+    def _bus_id(self):
         import torch
-        try:
-            p = torch.cuda.get_device_properties(self.cuda_index)
-            bus = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
-            return nv.nvmlDeviceGetHandleByPciBusId(bus)
-        except Exception:
-            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
+        p = torch.cuda.get_device_properties(self.cuda_index)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
 
-    def _run(self):
-        try:
-            import pynvml as nv
-            nv.nvmlInit()
-        except Exception as e:  # no NVML: the summary says so
-            self.error = f"nvml unavailable: {e}"
-            return
-        try:
-            h = self._handle(nv)
-            mx = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
-            while not self._stop.is_set():
-                sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = line.split()
+            if len(parts) == 4 and self._on:
                 try:
-                    pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
-                except Exception:
-                    pw = None
-                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.samples.append((sm, mx, pw, bits))
-                self._stop.wait(self.period)
-        except Exception as e:
-            self.error = f"nvml sampling failed: {e}"
-        finally:
-            try:
-                nv.nvmlShutdown()
-            except Exception:
-                pass
+                    pw = float(parts[2])
+                    self.samples.append((int(parts[0]), int(parts[1]),
+                                         pw if pw >= 0 else None, int(parts[3])))
+                except ValueError:
+                    pass
 
-    def __enter__(self):
-        self._thread = threading.Thread(target=self._run, daemon=True)
-        self._thread.start()
+    def start(self):
+        """Launch the sampler (its first samples arrive after it imports NVML)."""
+        import subprocess
+        try:
+            self.proc = subprocess.Popen(
+                [sys.executable, "-c", _SAMPLER, self._bus_id(), str(self.cuda_index),
+                 str(self.period)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError as e:
+            self.error = f"sampler did not start: {e}"
+            return self
+        self._reader = threading.Thread(target=self._read, daemon=True)
+        self._reader.start()
         return self
 
-    def __exit__(self, *exc):
-        self._stop.set()
-        if self._thread is not None:
-            self._thread.join(timeout=5)
-        return False
+    def record(self, on):
+        """Keep samples only while `on` (the warm-up and the timed region)."""
+        self._on = on
+
+    def stop(self):
+        self._on = False
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self._reader is not None:
+            self._reader.join(timeout=5)
 
     def summary(self):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
-                    "source": "nvml", "error": self.error}
-        import pynvml as nv
+                    "source": "nvml", "error": self.error or "no samples"}
+        try:
+            import pynvml as nv
+            consts = [(n, getattr(nv, c, 0)) for n, c in self.REASONS]
+        except ImportError:
+            consts = []
         reasons = set()
         for *_, bits in self.samples:
-            for name, const in self.REASONS:
-                if bits & getattr(nv, const, 0):
+            for name, c in consts:
+                if bits & c:
                     reasons.add(name)
         power = [s[2] for s in self.samples if s[2] is not None]
         return {"sm_mhz": statistics.median(s[0] for s in self.samples),
@@ -162,7 +191,7 @@ class ClockSampler:
                 "sm_max_mhz": max(s[1] for s in self.samples),
                 "power_w_median": round(statistics.median(power), 1) if power else None,
                 "reasons": sorted(reasons), "samples": len(self.samples),
-                "source": "nvml, 20 ms period, warm-up and timed region"}
+                "source": "nvml in a separate process, 2 ms period, warm-up and timed region"}
 
 
 def dist_setup(n_gpus, backend=None):
@@ -242,7 +271,9 @@ def run_ours(args):
 
     # Clocks are sampled from the warm-up on, so that even a short timed
     # region sees several samples of the loaded GPU.
-    clk = ClockSampler(local).__enter__()
+    clk = ClockSampler(local).start()
+    time.sleep(1.0)  # the sampler imports NVML before its first sample
+    clk.record(True)
     for _ in range(args.warmup):
         fwd()
         bwd()
@@ -264,7 +295,7 @@ def run_ours(args):
             ev[s][2].record(stream)
         t1.record(stream)
         torch.cuda.synchronize()
-    clk.__exit__(None, None, None)
+    clk.stop()
     fa.sync_status(dev)
     total_ms = t0.elapsed_time(t1)
     fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
