@@ -780,38 +780,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0 && ld_shared_volatile(abort_addr)) atomicOr(p.status, 1u);
 }
 
-// Work-item counters for the dynamic scheduler, one per launch in flight
-// (a launch takes the next slot and clears it on its stream first).
-constexpr int kSchedSlots = 64;
-__device__ unsigned int g_fwd_sched[kSchedSlots];
-
-unsigned int* sched_slot() {
-  static unsigned int* base[64] = {};
-  static unsigned int ticket = 0;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!base[dev]) {
-    void* a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_fwd_sched) != cudaSuccess) return nullptr;
-    base[dev] = static_cast<unsigned int*>(a);
-  }
-  const unsigned int t = __atomic_fetch_add(&ticket, 1u, __ATOMIC_RELAXED);
-  return base[dev] + (t % kSchedSlots);
-}
-
-int sm_count() {
-  static int count[64] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (count[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
-      n = 148;
-    count[dev] = n;
-  }
-  return count[dev];
-}
-
 }  // namespace
 
 template <int D>
@@ -847,7 +815,7 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   const int64_t kv_bytes = int64_t(2) * p.Sk * p.D * 2;
   int group = int((int64_t(128) << 20) / (kv_bytes > 0 ? kv_bytes : 1));
   group = group < 1 ? 1 : (group > p.B * p.N ? p.B * p.N : group);
-  unsigned int* sched = sched_slot();
+  unsigned int* sched = work_counter();
   if (!sched) return cudaErrorUnknown;
   if ((e = cudaMemsetAsync(sched, 0, sizeof(unsigned int), st)) != cudaSuccess) return e;
   fwd_bf16_sm100<D><<<grid, kThreads, C::kSmemBytes, st>>>(

@@ -26,6 +26,11 @@ cudaError_t launch_bwd_bf16_sm100(const Problem& p, const void* q,
                                   const float* delta, float* dq_acc, void* dk,
                                   void* dv, cudaStream_t st);
 
+// Dynamic scheduler of the persistent kernels (sched.cu): a cleared-per-
+// launch work counter (the caller clears it on its stream) and the SM count.
+unsigned int* work_counter();
+int sm_count();
+
 // Helpers (aux.cu).  is_bf16 selects the element type of the tensors.
 cudaError_t launch_bwd_pre(const Problem& p, bool is_bf16, const void* out,
                            const void* dout, float* delta, float* dq_acc,
