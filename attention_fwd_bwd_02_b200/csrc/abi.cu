@@ -35,8 +35,9 @@ fa_status check_shape(const fa_shape* s) {
     return FA_ERR_INVALID_ARG;
   if (s->layout != FA_LAYOUT_BNSD && s->layout != FA_LAYOUT_BSH)
     return FA_ERR_INVALID_ARG;
-  if (s->dtype != FA_F32 && s->dtype != FA_BF16) return FA_ERR_INVALID_ARG;
-  if (s->dtype == FA_BF16 && s->D != 64 && s->D != 128) return FA_ERR_UNSUPPORTED;
+  if (s->dtype != FA_F32 && s->dtype != FA_BF16 && s->dtype != FA_F16)
+    return FA_ERR_INVALID_ARG;
+  if (s->dtype != FA_F32 && s->D != 64 && s->D != 128) return FA_ERR_UNSUPPORTED;
   if (s->dtype == FA_F32 && s->D > 128) return FA_ERR_UNSUPPORTED;
   if (s->B > 65535 || s->N > 65535) return FA_ERR_UNSUPPORTED;
   return FA_OK;
@@ -56,6 +57,7 @@ fa_status make_problem(const fa_shape* s, const fa_pse* pse, const fa_mask* m,
   q.Sk = s->Sk;
   q.D = s->D;
   q.layout = s->layout;
+  q.f16 = s->dtype == FA_F16 ? 1u : 0u;
   const int64_t H = int64_t(s->N) * s->D;
   if (s->layout == FA_LAYOUT_BNSD) {
     q.q_sb = int64_t(s->N) * s->Sq * s->D;
@@ -142,7 +144,12 @@ fa_status cuda_status(cudaError_t e) {
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-size_t elem_size(const fa_shape* s) { return s->dtype == FA_BF16 ? 2 : 4; }
+size_t elem_size(const fa_shape* s) { return s->dtype == FA_F32 ? 4 : 2; }
+
+// Element type of the tensors for the helper kernels.
+fa::Elem elem_of(const fa_shape* s) {
+  return s->dtype == FA_F32 ? fa::Elem::kF32 : (s->dtype == FA_F16 ? fa::Elem::kF16 : fa::Elem::kBF16);
+}
 
 }  // namespace
 
@@ -176,7 +183,7 @@ fa_status run_fwd(const fa_shape* shape, const void* q, const void* k,
   fa_status st = make_problem(shape, pse, mask, scale, keep_prob, &p);
   if (st != FA_OK) return st;
   p.debug_flags = debug_flags;
-  if (debug_flags && shape->dtype != FA_BF16) return FA_ERR_UNSUPPORTED;
+  if (debug_flags && shape->dtype == FA_F32) return FA_ERR_UNSUPPORTED;
   if (p.B == 0 || p.N == 0 || p.Sq == 0) return FA_OK;  // nothing to write
   p.status = status_word();
   if (!p.status) return cuda_status(cudaErrorNoDevice);
@@ -185,12 +192,12 @@ fa_status run_fwd(const fa_shape* shape, const void* q, const void* k,
       (reinterpret_cast<uintptr_t>(lse) & 3u))
     return FA_ERR_INVALID_ARG;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  const bool bf16 = shape->dtype == FA_BF16;
+  const bool tc = shape->dtype != FA_F32;  // tensor-core path
   cudaError_t e;
   if (p.Sk == 0)
-    e = fa::launch_fill_empty_rows(p, bf16, out, lse, cs);
-  else if (bf16)
-    e = fa::launch_fwd_bf16_sm100(p, q, k, v, out, lse, cs);
+    e = fa::launch_fill_empty_rows(p, elem_of(shape), out, lse, cs);
+  else if (tc)
+    e = fa::launch_fwd_sm100(p, q, k, v, out, lse, cs);
   else
     e = fa::launch_fwd_f32(p, q, k, v, out, lse, cs);
   return cuda_status(e);
@@ -264,15 +271,15 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
   float* dq_acc = static_cast<float*>(workspace);
   float* delta = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                           round_up(rows * p.D * sizeof(float), 256));
-  const bool bf16 = shape->dtype == FA_BF16;
-  cudaError_t e = fa::launch_bwd_pre(p, bf16, out, dout, delta, dq_acc, cs);
+  const bool tc = shape->dtype != FA_F32;  // tensor-core path
+  cudaError_t e = fa::launch_bwd_pre(p, elem_of(shape), out, dout, delta, dq_acc, cs);
   if (e == cudaSuccess) {
-    if (bf16)
-      e = fa::launch_bwd_bf16_sm100(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, cs);
+    if (tc)
+      e = fa::launch_bwd_sm100(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, cs);
     else
       e = fa::launch_bwd_f32(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, cs);
   }
-  if (e == cudaSuccess) e = fa::launch_bwd_post(p, bf16, dq_acc, dq, cs);
+  if (e == cudaSuccess) e = fa::launch_bwd_post(p, elem_of(shape), dq_acc, dq, cs);
   return cuda_status(e);
 }
 

@@ -8,6 +8,7 @@
 //     layer 2, with a 2x2 allow table).
 // All are grid-strided, 16-byte vectorised where the layout allows.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -22,7 +23,9 @@ __device__ __forceinline__ float to_f(float x) { return x; }
 __device__ __forceinline__ float to_f(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
+__device__ __forceinline__ float to_f(__half x) { return __half2float(x); }
 __device__ __forceinline__ void from_f(float v, float* dst) { *dst = v; }
+__device__ __forceinline__ void from_f(float v, __half* dst) { *dst = __float2half_rn(v); }
 __device__ __forceinline__ void from_f(float v, __nv_bfloat16* dst) {
   *dst = __float2bfloat16_rn(v);
 }
@@ -37,6 +40,20 @@ __device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
   const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&u.x);
   const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&u.y);
   return make_float4(__low2float(a), __high2float(a), __low2float(b), __high2float(b));
+}
+__device__ __forceinline__ float4 load4(const __half* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+__device__ __forceinline__ void store4(__half* p, float4 v) {
+  __half2 a = __floats2half2_rn(v.x, v.y);
+  __half2 b = __floats2half2_rn(v.z, v.w);
+  uint2 u;
+  u.x = *reinterpret_cast<uint32_t*>(&a);
+  u.y = *reinterpret_cast<uint32_t*>(&b);
+  *reinterpret_cast<uint2*>(p) = u;
 }
 __device__ __forceinline__ void store4(float* p, float4 v) {
   *reinterpret_cast<float4*>(p) = v;
@@ -144,6 +161,25 @@ __device__ __forceinline__ void load16(const __nv_bfloat16* p, float (&v)[8]) {
     v[2 * k] = __uint_as_float(w[k] << 16);
     v[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
   }
+}
+__device__ __forceinline__ void load16(const __half* p, float (&v)[8]) {
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w[k]));
+    v[2 * k] = f.x;
+    v[2 * k + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void store16(__half* p, const float (&v)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const __half2 h2 = __floats2half2_rn(v[2 * k], v[2 * k + 1]);
+    w[k] = *reinterpret_cast<const uint32_t*>(&h2);
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 __device__ __forceinline__ void store16(float* p, const float (&v)[4]) {
   *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
@@ -299,22 +335,26 @@ int grid_for(int64_t work, int per_block) {
 
 }  // namespace
 
-cudaError_t launch_fill_empty_rows(const Problem& p, bool is_bf16, void* out,
-                                   float* lse, cudaStream_t st) {
+cudaError_t launch_fill_empty_rows(const Problem& p, Elem elem, void* out, float* lse,
+                                   cudaStream_t st) {
   const int64_t rows = int64_t(p.B) * p.N * p.Sq;
   const int g = grid_for(rows, 256);
-  if (is_bf16)
+  if (elem == Elem::kBF16)
     fill_empty_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
         p, static_cast<__nv_bfloat16*>(out), lse);
+  else if (elem == Elem::kF16)
+    fill_empty_kernel<__half><<<g, 256, 0, st>>>(p, static_cast<__half*>(out), lse);
   else
     fill_empty_kernel<float><<<g, 256, 0, st>>>(p, static_cast<float*>(out), lse);
   return cudaGetLastError();
 }
 
+namespace {
+
 // Lanes per row of the vectorised kernels (16-byte chunks), 0 if the row
 // does not split into a power-of-two number of chunks of at most 32.
-int lanes_per_row(const Problem& p, bool is_bf16) {
-  const int ve = is_bf16 ? 8 : 4;
+int lanes_per_row(const Problem& p, Elem elem) {
+  const int ve = elem == Elem::kF32 ? 4 : 8;
   if (p.D % ve != 0) return 0;
   const int lpr = p.D / ve;
   return (lpr == 8 || lpr == 16 || lpr == 32) ? lpr : 0;
@@ -341,45 +381,45 @@ cudaError_t post_vec(const Problem& p, int lpr, int g, const float* dq_acc, void
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_pre(const Problem& p, bool is_bf16, const void* out,
-                           const void* dout, float* delta, float* dq_acc,
-                           cudaStream_t st) {
+template <typename T>
+cudaError_t pre_any(const Problem& p, const void* out, const void* dout, float* delta,
+                    float* dq_acc, int lpr, cudaStream_t st) {
   const int64_t rows = int64_t(p.B) * p.N * p.Sq;
-  const int lpr = lanes_per_row(p, is_bf16);
   if (lpr) {
     // 8 warps per block, each covering 2 passes of 32 / lpr rows.
-    const int g = grid_for(rows, 8 * 2 * (32 / lpr));
-    return is_bf16 ? pre_vec<__nv_bfloat16>(p, lpr, g, out, dout, delta, dq_acc, st)
-                   : pre_vec<float>(p, lpr, g, out, dout, delta, dq_acc, st);
+    return pre_vec<T>(p, lpr, grid_for(rows, 8 * 2 * (32 / lpr)), out, dout, delta, dq_acc, st);
   }
-  const int g = grid_for(rows, 8);
-  if (is_bf16)
-    bwd_pre_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
-        p, static_cast<const __nv_bfloat16*>(out),
-        static_cast<const __nv_bfloat16*>(dout), delta, dq_acc);
-  else
-    bwd_pre_kernel<float><<<g, 256, 0, st>>>(
-        p, static_cast<const float*>(out), static_cast<const float*>(dout),
-        delta, dq_acc);
+  bwd_pre_kernel<T><<<grid_for(rows, 8), 256, 0, st>>>(
+      p, static_cast<const T*>(out), static_cast<const T*>(dout), delta, dq_acc);
   return cudaGetLastError();
 }
 
-cudaError_t launch_bwd_post(const Problem& p, bool is_bf16,
-                            const float* dq_acc, void* dq, cudaStream_t st) {
+template <typename T>
+cudaError_t post_any(const Problem& p, const float* dq_acc, void* dq, int lpr,
+                     cudaStream_t st) {
   const int64_t rows = int64_t(p.B) * p.N * p.Sq;
-  const int lpr = lanes_per_row(p, is_bf16);
-  if (lpr) {
-    const int g = grid_for(rows, 8 * 2 * (32 / lpr));
-    return is_bf16 ? post_vec<__nv_bfloat16>(p, lpr, g, dq_acc, dq, st)
-                   : post_vec<float>(p, lpr, g, dq_acc, dq, st);
-  }
-  const int g = grid_for(rows, 8);
-  if (is_bf16)
-    bwd_post_kernel<__nv_bfloat16><<<g, 256, 0, st>>>(
-        p, dq_acc, static_cast<__nv_bfloat16*>(dq));
-  else
-    bwd_post_kernel<float><<<g, 256, 0, st>>>(p, dq_acc, static_cast<float*>(dq));
+  if (lpr) return post_vec<T>(p, lpr, grid_for(rows, 8 * 2 * (32 / lpr)), dq_acc, dq, st);
+  bwd_post_kernel<T><<<grid_for(rows, 8), 256, 0, st>>>(p, dq_acc, static_cast<T*>(dq));
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_pre(const Problem& p, Elem elem, const void* out,
+                           const void* dout, float* delta, float* dq_acc,
+                           cudaStream_t st) {
+  const int lpr = lanes_per_row(p, elem);
+  if (elem == Elem::kBF16) return pre_any<__nv_bfloat16>(p, out, dout, delta, dq_acc, lpr, st);
+  if (elem == Elem::kF16) return pre_any<__half>(p, out, dout, delta, dq_acc, lpr, st);
+  return pre_any<float>(p, out, dout, delta, dq_acc, lpr, st);
+}
+
+cudaError_t launch_bwd_post(const Problem& p, Elem elem, const float* dq_acc, void* dq,
+                            cudaStream_t st) {
+  const int lpr = lanes_per_row(p, elem);
+  if (elem == Elem::kBF16) return post_any<__nv_bfloat16>(p, dq_acc, dq, lpr, st);
+  if (elem == Elem::kF16) return post_any<__half>(p, dq_acc, dq, lpr, st);
+  return post_any<float>(p, dq_acc, dq, lpr, st);
 }
 
 cudaError_t launch_tile_map(const Problem& p, uint8_t* tile_map,

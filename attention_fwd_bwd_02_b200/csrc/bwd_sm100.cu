@@ -1,4 +1,5 @@
-// bwd_sm100.cu -- bf16 attention backward on the 5th-generation tensor cores.
+// bwd_sm100.cu -- bf16 / fp16 attention backward on the 5th-generation tensor
+// cores.
 //
 // Gradients of sum(dO * O) for O = Softmax(Q K^T * scale + mask + alibi) V.
 // The probabilities are recomputed from the forward's per-row log-sum-exp
@@ -11,8 +12,8 @@
 // that can see it.  Everything is computed transposed, keys on the TMEM
 // lanes.  Two TMEM buffers of 128 columns alternate between query tiles:
 //   S^T = K Q^T  (SS) -> cols [0, 64),  dP^T = V dO^T (SS) -> cols [64, 128)
-//   the softmax warps then write P^T (bf16) to cols [0, 32) and dS^T (bf16)
-//   to cols [32, 64), and dQ^T = K^T dS^T (SS, dS^T staged in shared memory)
+//   the softmax warps then write P^T and dS^T (operand type) to cols [0, 32)
+//   and [32, 64), and dQ^T = K^T dS^T (SS, dS^T staged in shared memory)
 //   lands in cols [64, 128).
 //   dV += P^T dO  (P^T from TMEM) and dK += dS^T Q (dS^T from TMEM)
 //   accumulate in cols [256, 256+D) and [256+D, 256+2D).
@@ -43,8 +44,8 @@ constexpr int kBN = 128;  // keys per CTA
 constexpr int kBM = 64;   // query rows per step
 constexpr int kThreads = 512;
 constexpr int kTmemCols = 512;
-constexpr int kKeyBox = 128 * 128;  // 128 rows x 64 cols bf16
-constexpr int kQBox = 64 * 128;     // 64 rows x 64 cols bf16
+constexpr int kKeyBox = 128 * 128;  // 128 rows x 64 cols, 16-bit
+constexpr int kQBox = 64 * 128;     // 64 rows x 64 cols, 16-bit
 constexpr int kColP = 0, kColDS = 32, kColDQ = 64, kColAcc = 256;
 // Register split.  Launch: 512 threads x 128 = 65536 registers.  After the
 // split: 2 softmax warpgroups x 128 x 168 + dQ warpgroup x 128 x 88 + control
@@ -67,7 +68,7 @@ struct BwdCfg {
   static constexpr int kSmemV = kSmemK + kKTile;
   static constexpr int kSmemQ = kSmemV + kKTile;                 // [stage]
   static constexpr int kSmemDO = kSmemQ + kStages * kQTile;      // [stage]
-  static constexpr int kSmemDS = kSmemDO + kStages * kQTile;     // [2] 128 x 64 bf16
+  static constexpr int kSmemDS = kSmemDO + kStages * kQTile;     // [2] 128 x 64, 16-bit
   // dQ staging: per dQ warp one box of 32 rows x (D / 4) fp32 columns; a
   // query tile goes out as two such boxes.
   static constexpr int kDqCols = D / 4;
@@ -144,15 +145,16 @@ __device__ __forceinline__ int count_qtiles(const Problem& p, const KeyCtx& c) {
 // First dQ column owned by dQ warp wq.
 __device__ __forceinline__ int col0_dq(int D, int wq) { return wq * (D / 4); }
 
-template <int D>
+// kF16 selects fp16 operands (Q, K, V, dO, P, dS, dK, dV); bf16 otherwise.
+template <int D, bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
-    bwd_bf16_sm100(const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_do,
-                   const __grid_constant__ CUtensorMap tm_dq, const Problem p,
-                   const float* __restrict__ lse, const float* __restrict__ delta,
-                   __nv_bfloat16* __restrict__ dk, __nv_bfloat16* __restrict__ dv) {
+    bwd_sm100(const __grid_constant__ CUtensorMap tm_q,
+              const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v,
+              const __grid_constant__ CUtensorMap tm_do,
+              const __grid_constant__ CUtensorMap tm_dq, const Problem p,
+              const float* __restrict__ lse, const float* __restrict__ delta,
+              uint16_t* __restrict__ dk, uint16_t* __restrict__ dv) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -251,9 +253,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else if (warp == 13) {
       // ---------------------------------------------------------- MMA
       if (elect_one()) {
-        constexpr uint32_t id_s = idesc_bf16_f32(128, kBM, 0, 0);  // S^T, dP^T
-        constexpr uint32_t id_kv = idesc_bf16_f32(128, D, 0, 1);   // dV, dK
-        constexpr uint32_t id_q = idesc_bf16_f32(D, kBM, 1, 1);    // dQ^T
+        constexpr uint32_t id_s = idesc_f32acc(128, kBM, 0, 0, kF16);  // S^T, dP^T
+        constexpr uint32_t id_kv = idesc_f32acc(128, D, 0, 1, kF16);   // dV, dK
+        constexpr uint32_t id_q = idesc_f32acc(D, kBM, 1, 1, kF16);    // dQ^T
                 const int n_tiles = count_qtiles(p, c);
         bool ok = mbar_wait_s(BAR(C::bKvFull), 0, abort_addr);
         // S^T = K Q^T and dP^T = V dO^T of step n into buffer n % 2.
@@ -469,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < kBM; e += 2) {
           pf[e] = ex2_approx(__uint_as_float(sr[e >> 5][e & 31]));
           pf[e + 1] = ex2_approx(__uint_as_float(sr[e >> 5][(e & 31) + 1]));
-          pk[e >> 1] = pack_bf16x2(pf[e], pf[e + 1]);
+          pk[e >> 1] = pack_h2<kF16>(pf[e], pf[e + 1]);
         }
         tmem_st32(tb + kColP, pk);
       }
@@ -488,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     f2_pack(nd.x, nd.y));
           float s0, s1;
           f2_unpack(fmul2(t2, f2_pack(pf[cc], pf[cc + 1])), s0, s1);
-          dsk[cc >> 1] = pack_bf16x2(s0, s1);
+          dsk[cc >> 1] = pack_h2<kF16>(s0, s1);
         }
       }
       tmem_st32(tb + kColDS, dsk);
@@ -521,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool real = j < p.Sk;
     const int col = g == 0 ? C::kColDV : C::kColDK;
     const float mul = g == 0 ? 1.f : p.scale;
-    __nv_bfloat16* dst_row =
+    uint16_t* dst_row =
         (g == 0 ? dv : dk) + c.b * p.k_sb + c.h * p.k_sh + int64_t(j) * p.k_ss;
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
@@ -536,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 16; ++e) {
           const float x0 = have ? __uint_as_float(a[2 * e]) * mul : 0.f;
           const float x1 = have ? __uint_as_float(a[2 * e + 1]) * mul : 0.f;
-          w[e] = pack_bf16x2(x0, x1);
+          w[e] = pack_h2<kF16>(x0, x1);
         }
         uint4* dst = reinterpret_cast<uint4*>(dst_row + cc * 32);
 #pragma unroll
@@ -555,7 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0 && ld_shared_volatile(abort_addr)) atomicOr(p.status, 1u);
 }
 
-template <int D>
+template <int D, bool kF16>
 cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
                          const void* v, const void* dout, const float* lse,
                          const float* delta, float* dq_acc, void* dk, void* dv,
@@ -570,37 +572,40 @@ cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
   if ((e = make_f32_rows_map(&tdq, dq_acc, p.D, p.Sq, int64_t(p.B) * p.N, C::kDqCols,
                              C::kDqRows)) != cudaSuccess)
     return e;
-  e = cudaFuncSetAttribute(bwd_bf16_sm100<D>,
+  e = cudaFuncSetAttribute(bwd_sm100<D, kF16>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (e != cudaSuccess) return e;
   // The register split (setmaxnreg) draws on the launch allocation of
   // 65536 / kThreads registers per thread; a build with fewer would leave
   // the increase waiting.
-  static int regs_ok[2] = {0, 0};
-  if (!regs_ok[D == 128]) {
+  static int regs_ok[2][2] = {{0, 0}, {0, 0}};
+  if (!regs_ok[kF16][D == 128]) {
     cudaFuncAttributes fa_attr;
-    if ((e = cudaFuncGetAttributes(&fa_attr, bwd_bf16_sm100<D>)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa_attr, bwd_sm100<D, kF16>)) != cudaSuccess) return e;
     if (fa_attr.numRegs * kThreads < 2 * 128 * int(kRegsSoftmax) + 128 * int(kRegsDq) +
                                          128 * int(kRegsControl))
       return cudaErrorInvalidConfiguration;
-    regs_ok[D == 128] = 1;
+    regs_ok[kF16][D == 128] = 1;
   }
   dim3 grid((p.Sk + kBN - 1) / kBN, p.N, p.B);
-  bwd_bf16_sm100<D><<<grid, kThreads, C::kSmemBytes, st>>>(
-      tq, tk, tv, tdo, tdq, p, lse, delta, static_cast<__nv_bfloat16*>(dk),
-      static_cast<__nv_bfloat16*>(dv));
+  bwd_sm100<D, kF16><<<grid, kThreads, C::kSmemBytes, st>>>(
+      tq, tk, tv, tdo, tdq, p, lse, delta, static_cast<uint16_t*>(dk),
+      static_cast<uint16_t*>(dv));
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_bwd_bf16_sm100(const Problem& p, const void* q,
-                                  const void* k, const void* v,
-                                  const void* dout, const float* lse,
-                                  const float* delta, float* dq_acc, void* dk,
-                                  void* dv, cudaStream_t st) {
-  if (p.D == 64) return launch_bwd_d<64>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
-  if (p.D == 128) return launch_bwd_d<128>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
+cudaError_t launch_bwd_sm100(const Problem& p, const void* q, const void* k,
+                             const void* v, const void* dout, const float* lse,
+                             const float* delta, float* dq_acc, void* dk, void* dv,
+                             cudaStream_t st) {
+  if (p.D == 64)
+    return p.f16 ? launch_bwd_d<64, true>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st)
+                 : launch_bwd_d<64, false>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
+  if (p.D == 128)
+    return p.f16 ? launch_bwd_d<128, true>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st)
+                 : launch_bwd_d<128, false>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
   return cudaErrorInvalidValue;
 }
 

@@ -27,6 +27,7 @@ struct Problem {
   const int32_t* ids;       // modality ids [B][Sk]
   uint32_t allow_bits;      // bit (2*id_q + id_k): allowed; bit 4: diagonal
   const float* slopes;      // ALiBi slopes [N] or null
+  uint32_t f16;             // tensor-core path: 1 = fp16 operands, 0 = bf16
   uint32_t debug_flags;     // test hooks, 0 in production (kDebug* below)
   unsigned int* status;     // device status word (bit 0: a wait timed out)
 };

@@ -1,4 +1,5 @@
-// fwd_sm100.cu -- bf16 attention forward on the 5th-generation tensor cores.
+// fwd_sm100.cu -- bf16 / fp16 attention forward on the 5th-generation tensor
+// cores.
 //
 // Computes out = Softmax(Q K^T * scale + mask + alibi) V and the per-row
 // log-sum-exp ("FlashAttentionScore fusion operator replacement guide",
@@ -16,7 +17,7 @@
 // Warp roles:
 //   warps 0-3 / 4-7  softmax of query tile 0 / 1: thread t owns query row t.
 //              Reads S from TMEM, applies scale / ALiBi / mask, updates the
-//              running max and sum, writes P (bf16) back into TMEM over S,
+//              running max and sum, writes P (operand type) back into TMEM over S,
 //              rescales O in TMEM when the running max grew by more than
 //              2^8, and at the end of an item writes O / l and the LSE.
 //   warp 8     TMA producer: both Q tiles per item, then K_j and V_j through
@@ -49,7 +50,7 @@ constexpr int kBM = 128;              // query rows per tile
 constexpr int kTiles = 2;             // query tiles per work item
 constexpr int kRows = kBM * kTiles;   // query rows per work item
 constexpr int kBN = 128;              // keys per tile
-constexpr int kBoxBytes = 128 * 128;  // one 128-row x 64-col bf16 box
+constexpr int kBoxBytes = 128 * 128;  // one 128-row x 64-col 16-bit box
 constexpr int kThreads = 384;         // 3 warpgroups
 constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only if max grows > 2^8
@@ -255,14 +256,14 @@ __device__ __forceinline__ int tile_class(const Problem& p, const Item& c, int t
   return cls;
 }
 
-template <int D>
+// kF16 selects fp16 operands (Q, K, V, P, out); bf16 otherwise.
+template <int D, bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
-    fwd_bf16_sm100(const __grid_constant__ CUtensorMap tm_q,
-                   const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const Problem p,
-                   __nv_bfloat16* __restrict__ out, float* __restrict__ lse,
-                   int q_blocks, int n_items, int group,
-                   unsigned int* __restrict__ sched) {
+    fwd_sm100(const __grid_constant__ CUtensorMap tm_q,
+              const __grid_constant__ CUtensorMap tm_k,
+              const __grid_constant__ CUtensorMap tm_v, const Problem p,
+              uint16_t* __restrict__ out, float* __restrict__ lse, int q_blocks,
+              int n_items, int group, unsigned int* __restrict__ sched) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -411,8 +412,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     } else if (warp == 9) {
       // ---------------------------------------------------------- MMA
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kBN, 0, 0);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+      constexpr uint32_t idesc_qk = idesc_f32acc(128, kBN, 0, 0, kF16);
+      constexpr uint32_t idesc_pv = idesc_f32acc(128, D, 0, 1, kF16);
       // Operand descriptors as low halves (start address + leading offset);
       // every operand here has an 8-row stride of 1024 B (common high half).
       // Q and K are K-major (64-column boxes); V is N-major with a box of
@@ -676,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           m_ref = mx;
           rescale = true;
         }
-        // P = 2^(x - m) in bf16, written over the S columns already read
+        // P = 2^(x - m) in the operand type, written over the S columns read
         // (keys 32q..32q+31 -> packed columns 16q..16q+15).
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t neg_m = f2_pack(-m_use, -m_use);
@@ -698,7 +699,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               p1 = ex2_approx(a1);
             }
             rs2[(e >> 1) & 3] = fadd2(rs2[(e >> 1) & 3], f2_pack(p0, p1));
-            pk[e >> 1] = pack_bf16x2(p0, p1);
+            pk[e >> 1] = pack_h2<kF16>(p0, p1);
           }
           tmem_st16(tS + q4 * 16, pk);
         }
@@ -738,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const bool empty = !(l > 0.f);
       const float inv = empty ? 0.f : 1.f / l;
-      __nv_bfloat16* orow = out + c.b * p.q_sb + c.h * p.q_sh + int64_t(i) * p.q_ss;
+      uint16_t* orow = out + c.b * p.q_sb + c.h * p.q_sh + int64_t(i) * p.q_ss;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t orr[32];
@@ -757,7 +758,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 16; ++e) {
             const float o0 = (have_o && !empty) ? __uint_as_float(orr[2 * e]) * inv : 0.f;
             const float o1 = (have_o && !empty) ? __uint_as_float(orr[2 * e + 1]) * inv : 0.f;
-            wv[e] = pack_bf16x2(o0, o1);
+            wv[e] = pack_h2<kF16>(o0, o1);
           }
           uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
@@ -782,7 +783,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <int D>
+template <int D, bool kF16>
 static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
                                 const void* v, void* out, float* lse,
                                 cudaStream_t st) {
@@ -792,18 +793,18 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   if ((e = make_operand_map(&tk, k, p, p.Sk, 128)) != cudaSuccess) return e;
   if ((e = make_operand_map(&tv, v, p, p.Sk, 128)) != cudaSuccess) return e;
   using C = FwdCfg<D>;
-  e = cudaFuncSetAttribute(fwd_bf16_sm100<D>,
+  e = cudaFuncSetAttribute(fwd_sm100<D, kF16>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmemBytes);
   if (e != cudaSuccess) return e;
   // The register split (setmaxnreg) draws on the launch allocation; a build
   // with fewer registers per thread would leave the increase waiting.
-  static int regs_ok[2] = {0, 0};
-  if (!regs_ok[D == 128]) {
+  static int regs_ok[2][2] = {{0, 0}, {0, 0}};
+  if (!regs_ok[kF16][D == 128]) {
     cudaFuncAttributes fa_attr;
-    if ((e = cudaFuncGetAttributes(&fa_attr, fwd_bf16_sm100<D>)) != cudaSuccess) return e;
+    if ((e = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16>)) != cudaSuccess) return e;
     if (fa_attr.numRegs < int(kRegsLaunch)) return cudaErrorInvalidConfiguration;
-    regs_ok[D == 128] = 1;
+    regs_ok[kF16][D == 128] = 1;
   }
   const int q_blocks = (p.Sq + kRows - 1) / kRows;
   const int64_t items = int64_t(q_blocks) * p.B * p.N;
@@ -818,17 +819,21 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   unsigned int* sched = work_counter();
   if (!sched) return cudaErrorUnknown;
   if ((e = cudaMemsetAsync(sched, 0, sizeof(unsigned int), st)) != cudaSuccess) return e;
-  fwd_bf16_sm100<D><<<grid, kThreads, C::kSmemBytes, st>>>(
-      tq, tk, tv, p, static_cast<__nv_bfloat16*>(out), lse, q_blocks, int(items), group,
+  fwd_sm100<D, kF16><<<grid, kThreads, C::kSmemBytes, st>>>(
+      tq, tk, tv, p, static_cast<uint16_t*>(out), lse, q_blocks, int(items), group,
       sched);
   return cudaGetLastError();
 }
 
-cudaError_t launch_fwd_bf16_sm100(const Problem& p, const void* q,
-                                  const void* k, const void* v, void* out,
-                                  float* lse, cudaStream_t st) {
-  if (p.D == 64) return launch_fwd_d<64>(p, q, k, v, out, lse, st);
-  if (p.D == 128) return launch_fwd_d<128>(p, q, k, v, out, lse, st);
+cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k,
+                             const void* v, void* out, float* lse,
+                             cudaStream_t st) {
+  if (p.D == 64)
+    return p.f16 ? launch_fwd_d<64, true>(p, q, k, v, out, lse, st)
+                 : launch_fwd_d<64, false>(p, q, k, v, out, lse, st);
+  if (p.D == 128)
+    return p.f16 ? launch_fwd_d<128, true>(p, q, k, v, out, lse, st)
+                 : launch_fwd_d<128, false>(p, q, k, v, out, lse, st);
   return cudaErrorInvalidValue;
 }
 

@@ -16,28 +16,29 @@ cudaError_t launch_bwd_f32(const Problem& p, const void* q, const void* k,
                            const float* delta, float* dq_acc, void* dk,
                            void* dv, cudaStream_t st);
 
-// bf16 tensor-core path (fwd_sm100.cu, bwd_sm100.cu).
-cudaError_t launch_fwd_bf16_sm100(const Problem& p, const void* q,
-                                  const void* k, const void* v, void* out,
-                                  float* lse, cudaStream_t st);
-cudaError_t launch_bwd_bf16_sm100(const Problem& p, const void* q,
-                                  const void* k, const void* v,
-                                  const void* dout, const float* lse,
-                                  const float* delta, float* dq_acc, void* dk,
-                                  void* dv, cudaStream_t st);
+// bf16 / fp16 tensor-core path (fwd_sm100.cu, bwd_sm100.cu); p.f16 selects
+// the operand type.
+cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k,
+                             const void* v, void* out, float* lse,
+                             cudaStream_t st);
+cudaError_t launch_bwd_sm100(const Problem& p, const void* q, const void* k,
+                             const void* v, const void* dout, const float* lse,
+                             const float* delta, float* dq_acc, void* dk,
+                             void* dv, cudaStream_t st);
 
 // Dynamic scheduler of the persistent kernels (sched.cu): a cleared-per-
 // launch work counter (the caller clears it on its stream) and the SM count.
 unsigned int* work_counter();
 int sm_count();
 
-// Helpers (aux.cu).  is_bf16 selects the element type of the tensors.
-cudaError_t launch_bwd_pre(const Problem& p, bool is_bf16, const void* out,
+// Helpers (aux.cu), for tensors of element type `elem`.
+enum class Elem { kF32, kBF16, kF16 };
+cudaError_t launch_bwd_pre(const Problem& p, Elem elem, const void* out,
                            const void* dout, float* delta, float* dq_acc,
                            cudaStream_t st);
-cudaError_t launch_bwd_post(const Problem& p, bool is_bf16,
-                            const float* dq_acc, void* dq, cudaStream_t st);
-cudaError_t launch_fill_empty_rows(const Problem& p, bool is_bf16, void* out,
+cudaError_t launch_bwd_post(const Problem& p, Elem elem, const float* dq_acc,
+                            void* dq, cudaStream_t st);
+cudaError_t launch_fill_empty_rows(const Problem& p, Elem elem, void* out,
                                    float* lse, cudaStream_t st);
 cudaError_t launch_tile_map(const Problem& p, uint8_t* tile_map,
                             cudaStream_t st);

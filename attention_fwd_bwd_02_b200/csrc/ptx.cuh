@@ -315,15 +315,19 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem,
       : "memory");
 }
 
-// Instruction descriptor of tcgen05.mma kind::f16 with bf16 A/B and fp32 D.
-// Bit layout: [4,6) D format (1 = f32), [7,10) A format (1 = bf16),
-// [10,13) B format (1 = bf16), 15 A major (1 = MN), 16 B major (1 = MN),
-// [17,23) N >> 3, [24,29) M >> 4.
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn,
-                                                      int b_mn) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(a_mn) << 15) |
-         (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) |
+// Instruction descriptor of tcgen05.mma kind::f16 with fp32 D and A/B both
+// bf16 (f16 = false) or both fp16 (f16 = true).
+// Bit layout: [4,6) D format (1 = f32), [7,10) A format (0 = f16,
+// 1 = bf16), [10,13) B format (same codes), 15 A major (1 = MN), 16 B major
+// (1 = MN), [17,23) N >> 3, [24,29) M >> 4.
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int a_mn, int b_mn,
+                                                    bool f16) {
+  return (1u << 4) | ((f16 ? 0u : 1u) << 7) | ((f16 ? 0u : 1u) << 10) |
+         (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) |
          (uint32_t(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
+  return idesc_f32acc(M, N, a_mn, b_mn, false);
 }
 
 // Shared-memory matrix descriptor for a 128-byte-swizzled operand.
@@ -533,6 +537,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+// Two fp32 -> packed f16x2 with round-to-nearest-even; `lo` in bits 0..15.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+// The operand type of the tensor-core kernels: fp16 when kF16, else bf16.
+template <bool kF16>
+__device__ __forceinline__ uint32_t pack_h2(float lo, float hi) {
+  return kF16 ? pack_f16x2(lo, hi) : pack_bf16x2(lo, hi);
 }
 
 }  // namespace fa

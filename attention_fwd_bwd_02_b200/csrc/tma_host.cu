@@ -36,7 +36,7 @@ cudaError_t make_operand_map(CUtensorMap* map, const void* base,
   EncodeTiledFn enc = get_encode();
   if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[3], strides[2];
-  const cuuint64_t esz = 2;  // bf16
+  const cuuint64_t esz = 2;  // bf16 or fp16
   if (p.layout == FA_LAYOUT_BSH) {
     dims[0] = cuuint64_t(p.N) * p.D;
     dims[1] = cuuint64_t(S);
@@ -52,7 +52,7 @@ cudaError_t make_operand_map(CUtensorMap* map, const void* base,
   }
   const cuuint32_t box[3] = {64u, cuuint32_t(box_rows), 1u};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+  CUresult r = enc(map, p.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
                    const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,

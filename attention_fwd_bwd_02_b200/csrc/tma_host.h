@@ -1,5 +1,5 @@
-// tma_host.h -- host-side construction of TMA tensor maps for the bf16
-// operands (Q, K, V, dO, ...).
+// tma_host.h -- host-side construction of TMA tensor maps for the bf16 /
+// fp16 operands (Q, K, V, dO, ...).
 #pragma once
 
 #include <cuda.h>
@@ -9,7 +9,8 @@
 
 namespace fa {
 
-// Tensor map over a bf16 operand with S rows per head, read as boxes of
+// Tensor map over a bf16 (p.f16 = 0) or fp16 (p.f16 = 1) operand with S
+// rows per head, read as boxes of
 // 64 columns x box_rows rows with 128-byte swizzle (the canonical K-major /
 // MN-major operand layout of tcgen05).  Coordinates (x, row, z):
 //   BNSD: x = column 0..D-1, z = b*N + h;   BSH: x = h*D + column, z = b.

@@ -26,7 +26,7 @@ TESTING_HEADER = os.path.join(os.path.dirname(_HERE), "include", "fa_testing.h")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 FA_LAYOUT_BNSD, FA_LAYOUT_BSH = 0, 1
-FA_F32, FA_BF16 = 0, 1
+FA_F32, FA_BF16, FA_F16 = 0, 1, 2
 FA_MASK_CAUSAL, FA_MASK_KV_PADDING, FA_MASK_BOOL, FA_MASK_MODALITY = 1, 2, 4, 8
 FA_PSE_NONE, FA_PSE_ALIBI = 0, 1
 FA_TILE_M = FA_TILE_N = 128
@@ -135,6 +135,8 @@ def _stream(t: torch.Tensor):
 def _dtype_code(dt):
     if dt == torch.bfloat16:
         return FA_BF16
+    if dt == torch.float16:
+        return FA_F16
     if dt == torch.float32:
         return FA_F32
     raise FaError(FA_ERR_UNSUPPORTED, f"dtype {dt}")

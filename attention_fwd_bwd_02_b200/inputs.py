@@ -3,7 +3,7 @@
 This module holds no attention arithmetic: it only draws random tensors and
 integer side inputs (padding lengths, modality ids, ALiBi slopes) on the CPU.
 Both the CUDA path and the fp64 oracle consume what it returns, so input
-rounding (fp32 -> bf16, round-to-nearest-even, done once here) is never
+rounding (fp32 -> bf16 or fp16, round-to-nearest-even, done once here) is never
 counted as kernel error.
 
 Workloads (the shapes and value distributions of the attention call sites on
@@ -114,7 +114,7 @@ def make_case(name, B, N, Sq, Sk, D, *, dtype=torch.bfloat16, layout="BNSD",
         n_text, n_image = modality
         assert n_text + n_image == Sq == Sk
         ids = modality_ids_text_image(B, n_text, n_image)
-    if dtype not in (torch.float32, torch.bfloat16):
+    if dtype not in (torch.float32, torch.bfloat16, torch.float16):
         raise ValueError(f"unsupported dtype {dtype}")
 
     def cast(t):

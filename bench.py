@@ -354,8 +354,8 @@ def run_ours(args):
     dominant = "bwd" if bwd_ms >= fwd_ms else "fwd"
 
     def roof(kind, tf, ms):
-        return {"kernel": "fa_fwd (fwd_bf16_sm100)" if kind == "fwd" else
-                "fa_bwd (bwd_pre + bwd_bf16_sm100 + bwd_post)",
+        return {"kernel": "fa_fwd (fwd_sm100)" if kind == "fwd" else
+                "fa_bwd (bwd_pre + bwd_sm100 + bwd_post)",
                 "bound": "tensor", "achieved": round(tf, 1), "peak": peak_burst,
                 "unit": "TFLOP/s", "frac": round(tf / peak_burst, 4),
                 "peak_kind": f"{pk_kind} bf16_tflops (burst)",

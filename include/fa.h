@@ -31,8 +31,9 @@
  *                      H = N * D and head h at columns h*D .. h*D+D-1.
  *    All contiguous, D innermost.  out, dq, dk, dv use the layout and dtype
  *    of q, k, v.  lse is always fp32 [B][N][Sq].
- *  - Dtypes: FA_BF16 (tensor-core path, D in {64, 128}) or FA_F32 (fp32 FMA
- *    path, 1 <= D <= 128).  Accumulation is fp32 in both.
+ *  - Dtypes: FA_BF16 or FA_F16 (tensor-core path, D in {64, 128}), or FA_F32
+ *    (fp32 FMA path, 1 <= D <= 128).  Accumulation is fp32 in all three; P
+ *    and dS enter the tensor core in the operand type.
  *  - Tensor pointers must be 16-byte aligned.
  */
 #ifndef FA_B200_H
@@ -54,7 +55,7 @@ typedef enum {
 } fa_status;
 
 typedef enum { FA_LAYOUT_BNSD = 0, FA_LAYOUT_BSH = 1 } fa_layout;
-typedef enum { FA_F32 = 0, FA_BF16 = 1 } fa_dtype;
+typedef enum { FA_F32 = 0, FA_BF16 = 1, FA_F16 = 2 } fa_dtype;
 
 /* Mask rules (bit flags, combinable).  A key j is visible to query i when
  * every active rule allows it.  Disallowed scores are -inf before the
@@ -119,7 +120,7 @@ typedef struct {
  *               FA_ERR_UNSUPPORTED.
  * Errors: FA_ERR_INVALID_ARG for null tensors, non-positive sizes, a
  * modality mask with Sq != Sk or a missing mask pointer; FA_ERR_UNSUPPORTED
- * for keep_prob != 1 or a bf16 head dim other than 64 / 128. */
+ * for keep_prob != 1 or a bf16 / fp16 head dim other than 64 / 128. */
 fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
                  const void* v, const fa_pse* pse, const fa_mask* mask,
                  float scale, float keep_prob, void* out, float* lse,

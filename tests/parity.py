@@ -2,7 +2,7 @@
 (via the C-ABI binding) and through the fp64 oracle, and compare.
 
 Tolerances (fixed by the problem statement of this operator):
-  bf16 in/out, fp32 accumulation : max|d| <= 2e-2 and mean|d| <= 2e-3
+  bf16 or fp16 in/out, fp32 accumulation : max|d| <= 2e-2 and mean|d| <= 2e-3
   fp32 path                      : max|d| <= 1e-4
   rows with no visible key       : out exactly 0, lse exactly -inf
 The same bounds are applied to the LSE.  For gradients of large workloads

@@ -62,6 +62,7 @@ def _fwd(L, shape, pse=None, mask=None, scale=0.125, keep_prob=1.0, ptr=FAKE):
 
 @pytest.mark.parametrize("kw,code", [
     (dict(D=96), fa.FA_ERR_UNSUPPORTED),          # bf16 head dim not 64/128
+    (dict(D=96, dtype=fa.FA_F16), fa.FA_ERR_UNSUPPORTED),  # fp16 likewise
     (dict(D=256, dtype=fa.FA_F32), fa.FA_ERR_UNSUPPORTED),
     (dict(D=0), fa.FA_ERR_INVALID_ARG),
     (dict(B=-1), fa.FA_ERR_INVALID_ARG),
