@@ -14,9 +14,6 @@
 
 namespace fa {
 
-// Upper bound of a single wait (ns).  Real waits last micro-seconds.
-constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
-
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -25,12 +22,6 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
-}
-
-__device__ __forceinline__ uint32_t lane_id() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%laneid;" : "=r"(r));
-  return r;
 }
 
 __device__ __forceinline__ bool elect_one() {
@@ -83,7 +74,21 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity);
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Makes initialised barriers visible to the async proxy (TMA, tcgen05).
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
 // Bounded wait on a barrier phase; the abort flag is a shared-memory word
 // (0 = running) that this wait raises on timeout and polls while waiting.
 __device__ __forceinline__ bool mbar_wait_s(uint32_t bar, uint32_t parity,
@@ -103,12 +108,16 @@ __device__ __forceinline__ bool mbar_wait_s(uint32_t bar, uint32_t parity,
     }
   }
 }
-__device__ __forceinline__ void umma_commit_s(uint32_t bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
-      "[%0];" ::"r"(bar)
-      : "memory");
+
+// Orders this thread's generic shared-memory writes before later reads of
+// the same memory by the async proxy (TMA, tcgen05).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
+
+// ---------------------------------------------------------------- TMA
+
+// 3-D tiled load global -> shared, completion counted on `bar` (bytes).
 __device__ __forceinline__ void tma_load_3d_s(uint32_t smem_dst, const CUtensorMap* m,
                                               uint32_t bar, int c0, int c1, int c2) {
   asm volatile(
@@ -117,119 +126,11 @@ __device__ __forceinline__ void tma_load_3d_s(uint32_t smem_dst, const CUtensorM
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
       : "memory");
 }
-__device__ __forceinline__ void tmem_alloc_s(uint32_t dst, uint32_t ncols) {
-  asm volatile(
-      "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
-      "r"(ncols)
-      : "memory");
-}
-
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
-               "r"(count)
-               : "memory");
-}
-
-// Makes initialised barriers visible to the async proxy (TMA, tcgen05).
-__device__ __forceinline__ void fence_barrier_init() {
-  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar,
-                                                      uint32_t bytes) {
-  asm volatile(
-      "mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(
-          smem_u32(bar)),
-      "r"(bytes)
-      : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, P;\n\t}"
-      : "=r"(ok)
-      : "r"(addr), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Waits for the phase of `bar` with the given parity to complete.  Returns
-// false (and raises *abort_flag) if it did not within the limit, or if
-// another role of the CTA has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          volatile int* abort_flag,
-                                          uint64_t limit_ns = kWaitLimitNs) {
-  const uint32_t a = smem_u32(bar);
-  if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t it = 0;
-  while (true) {
-    if (mbar_try_wait(a, parity)) return true;
-    if ((++it & 15u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort_flag = 1;
-        return false;
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------- TMA
-
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m))
                : "memory");
 }
 
-// 4-D tiled load global -> shared, completion counted on `bar` (bytes).
-__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* m,
-                                            uint64_t* bar, int c0, int c1,
-                                            int c2, int c3) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::"
-      "bytes [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1),
-      "r"(c2), "r"(c3)
-      : "memory");
-}
-
-// 3-D tiled load global -> shared, completion counted on `bar` (bytes).
-__device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m,
-                                            uint64_t* bar, int c0, int c1,
-                                            int c2) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::"
-      "bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1),
-      "r"(c2)
-      : "memory");
-}
-
-// Bulk (untiled) reduce-add of fp32 shared -> global; both addresses 16-byte
-// aligned, bytes a multiple of 16.
-__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst,
-                                                    const float* ssrc,
-                                                    uint32_t bytes) {
-  asm volatile(
-      "cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], "
-      "%2;" ::"l"(gdst),
-      "r"(smem_u32(ssrc)), "r"(bytes)
-      : "memory");
-}
 // 3-D tiled reduce-add shared -> global (fp32 add), bulk-group completion.
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m,
                                                   const void* smem_src, int c0,
@@ -247,19 +148,15 @@ __device__ __forceinline__ void bulk_commit_group() {
 __device__ __forceinline__ void bulk_wait_group_read0() {
   asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 }
-__device__ __forceinline__ void bulk_wait_group_read1() {
-  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-}
 __device__ __forceinline__ void bulk_wait_group0() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
 // ---------------------------------------------------------------- tcgen05
 
-__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+__device__ __forceinline__ void tmem_alloc_s(uint32_t dst, uint32_t ncols) {
   asm volatile(
-      "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-          smem_u32(dst_smem)),
+      "tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
       "r"(ncols)
       : "memory");
 }
@@ -279,39 +176,12 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-
 // Arrive (once) on `bar` when every tcgen05 op this thread issued so far
 // has completed.
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+__device__ __forceinline__ void umma_commit_s(uint32_t bar) {
   asm volatile(
       "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 "
-      "[%0];" ::"r"(smem_u32(bar))
-      : "memory");
-}
-
-// D[tmem] (+)= A[smem desc] * B[smem desc]
-__device__ __forceinline__ void umma_ss(uint32_t d_tmem, uint64_t adesc,
-                                        uint64_t bdesc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(
-          d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc]
-__device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem,
-                                        uint64_t bdesc, uint32_t idesc,
-                                        uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(
-          d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      "[%0];" ::"r"(bar)
       : "memory");
 }
 
@@ -326,34 +196,20 @@ __host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int a_mn, int 
          (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16) | (uint32_t(N >> 3) << 17) |
          (uint32_t(M >> 4) << 24);
 }
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
-  return idesc_f32acc(M, N, a_mn, b_mn, false);
-}
 
-// Shared-memory matrix descriptor for a 128-byte-swizzled operand.
-//   K-major : rows of 128 B (64 bf16 along K), 8-row atoms of 1024 B;
-//             sbo = distance between 8-row atoms, lbo unused (16).
+// Shared-memory matrix descriptor of a 128-byte-swizzled operand, as its two
+// 32-bit halves.
+//   K-major : rows of 128 B (64 16-bit elements along K), 8-row atoms of
+//             1024 B; sbo = distance between 8-row atoms, lbo unused (16).
 //   MN-major: 128 B runs along M/N, 8 K-rows per atom;
 //             lbo = distance between 64-element M/N runs,
 //             sbo = distance between 8-row K groups.
-// Bits: [0,14) addr >> 4, [16,30) lbo >> 4, [32,46) sbo >> 4,
+// 64-bit layout: [0,14) addr >> 4, [16,30) lbo >> 4, [32,46) sbo >> 4,
 // [46,48) version = 1, [61,64) layout (2 = SWIZZLE_128B).
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo,
-                                                uint32_t sbo) {
-  uint64_t d = 0;
-  d |= uint64_t((saddr >> 4) & 0x3FFFu);
-  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
-  d |= uint64_t((sbo >> 4) & 0x3FFFu) << 32;
-  d |= uint64_t(1) << 46;
-  d |= uint64_t(2) << 61;
-  return d;
-}
-
-// The same descriptor as two 32-bit halves.  The start address sits in the
-// low half (bits 0..13, address >> 4) and shared-window addresses stay below
-// 256 KB, so advancing an operand by `bytes` is `lo + (bytes >> 4)` with no
-// carry into the other fields.  The MMA warp keeps one low half per operand
-// base and adds compile-time offsets, which keeps MMA issue to a few
+// The start address sits in the low half and shared-window addresses stay
+// below 256 KB, so advancing an operand by `bytes` is `lo + (bytes >> 4)`
+// with no carry into the other fields.  The MMA warp keeps one low half per
+// operand base and adds compile-time offsets, which keeps MMA issue to a few
 // instructions.
 __device__ __forceinline__ uint32_t sdesc_lo(uint32_t saddr, uint32_t lbo) {
   return ((saddr >> 4) & 0x3FFFu) | (((lbo >> 4) & 0x3FFFu) << 16);
@@ -410,17 +266,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "r"(taddr));
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]),
-        "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]),
-        "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15])
-      : "r"(taddr));
-}
-
 // Waits for this thread's outstanding TMEM loads.  The registers are tied
 // through the asm so that no use of them can be scheduled before the wait.
 __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
@@ -433,16 +278,6 @@ __device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[32]) {
         "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
         "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
         "+r"(r[30]), "+r"(r[31])
-      :
-      : "memory");
-}
-__device__ __forceinline__ void tmem_ld_wait(uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]),
-        "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]),
-        "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-        "+r"(r[15])
       :
       : "memory");
 }
