@@ -67,18 +67,20 @@ def source_hash():
     return h.hexdigest()[:16]
 
 
-def committed_traffic():
-    """Per-launch DRAM bytes from the committed ncu summary, if it was taken
-    on the current kernel sources (else None)."""
+def committed_ncu():
+    """Per-launch figures from the committed ncu summary, if it was taken on
+    the current kernel sources (else empty): DRAM bytes per kernel call
+    ("kernels") and per kernel duration, DRAM GB/s and tensor-pipe activity
+    ("ncu")."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
     except (OSError, ValueError):
-        return {}
+        return {}, {}
     if d.get("source_hash") != source_hash():
-        return {}
-    return d.get("kernels", {})
+        return {}, {}
+    return d.get("kernels", {}), d.get("ncu", {})
 
 
 _SAMPLER = r"""
@@ -350,7 +352,7 @@ def run_ours(args):
     bwd_tf = BWD_FLOPS / (bwd_ms * 1e-3) / 1e12
     peak_burst = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
     peak_sust = pk.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
-    traffic = committed_traffic()
+    traffic, ncu = committed_ncu()
     dominant = "bwd" if bwd_ms >= fwd_ms else "fwd"
 
     def roof(kind, tf, ms):
@@ -363,7 +365,10 @@ def run_ours(args):
                 "frac_of_nominal_2250": round(tf / 2250.0, 4),
                 "ms_per_launch": round(ms, 4),
                 "algorithmic_flops": FWD_FLOPS if kind == "fwd" else BWD_FLOPS,
-                "traffic": traffic.get(kind)}
+                "traffic": traffic.get(kind),
+                "ncu": ({"fwd_sm100": ncu.get("fwd")} if kind == "fwd" else
+                        {"bwd_pre": ncu.get("bwd_pre"), "bwd_sm100": ncu.get("bwd_main"),
+                         "bwd_post": ncu.get("bwd_post")}) if ncu else None}
 
     cpu = cpu_baseline(args) if not args.no_cpu_baseline else None
     line = {
