@@ -485,6 +485,102 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def _allowed_pairs(case):
+    """Visible (query, key) pairs of a case, summed over (b, h), from its
+    integer side inputs (padding lengths, modality ids, causal rule)."""
+    import torch
+    B, N, Sq, Sk = case.B, case.N, case.Sq, case.Sk
+    total = 0
+    for b in range(B):
+        nk = Sk if case.kv_len is None else max(0, min(Sk, int(case.kv_len[b])))
+        vis = torch.zeros(Sq, Sk, dtype=torch.bool)
+        vis[:, :nk] = True
+        if case.causal:
+            vis &= torch.ones(Sq, Sk, dtype=torch.bool).tril()
+        if case.modality_ids is not None:
+            ids = case.modality_ids[b].long() & 1
+            allow = torch.tensor(case.allow, dtype=torch.bool)
+            rule = allow[ids[:, None], ids[None, :]]
+            if case.allow_diag:
+                rule |= torch.eye(Sq, Sk, dtype=torch.bool)
+            vis &= rule
+        total += int(vis.sum()) * N
+    return total
+
+
+def run_configs(args):
+    """Times fa_fwd and fa_fwd + fa_bwd on every workload of the source pages
+    (one JSON line each, after the main line's format): nominal and
+    allowed-pair TFLOP/s, GB/s on the algorithmic bytes, and the fraction of
+    the measured peak.  HBM-bound workloads are timed with L2 flushed
+    between repetitions (a 256 MB write)."""
+    import statistics as st
+    import torch
+    from attention_fwd_bwd_02_b200 import fa
+    from attention_fwd_bwd_02_b200 import inputs as I
+    pk, pk_kind = peaks()
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    cases = [("1", I.config1(), False), ("2", I.config2(), False),
+             ("3a", I.config3(24), True), ("3b", I.config3(320), True),
+             ("4a", I.config4(256), True), ("4b", I.config4(512), True)]
+    cases += [(f"5 S={s} D={d}", I.config5(s, d), s <= 1024) for s, d in I.CONFIG5_SWEEP]
+    for label, c, do_flush in cases:
+        dev = {n: (None if getattr(c, n) is None else getattr(c, n).cuda())
+               for n in ("q", "k", "v", "dout")}
+        kw = dict(pse=None if c.slopes is None else c.slopes.cuda(), scale=c.scale,
+                  causal=c.causal,
+                  padding_kv_len=None if c.kv_len is None else c.kv_len.cuda())
+        if c.modality_ids is not None:
+            kw.update(modality_ids=c.modality_ids.cuda(), allow=c.allow, allow_diag=c.allow_diag)
+        q, k, v, do = dev["q"], dev["k"], dev["v"], dev["dout"]
+        out, lse = fa.fwd(q, k, v, c.N, c.layout, **kw)
+        ws = torch.empty(fa.bwd_workspace_size(fa.make_shape(q, k, c.N, c.layout)),
+                         dtype=torch.uint8, device="cuda")
+        fwd = lambda: fa.fwd(q, k, v, c.N, c.layout, out=out, lse=lse, **kw)
+        bwd = lambda: fa.bwd(q, k, v, out, do, lse, c.N, c.layout, workspace=ws, **kw)
+
+        def timed(fn, reps=30, warm=10):
+            for _ in range(warm):
+                fn()
+            ts = []
+            for _ in range(reps):
+                if do_flush:
+                    flush.fill_(1)
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                fn()
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1))
+            return st.median(ts)
+
+        f_ms = timed(fwd)
+        b_ms = timed(bwd)
+        fa.sync_status()
+        nominal = 4.0 * c.B * c.N * c.Sq * c.Sk * c.D / (2.0 if c.causal else 1.0)
+        allowed = 4.0 * c.D * _allowed_pairs(c)
+        esz = q.element_size()
+        rows_q, rows_k = c.B * c.N * c.Sq, c.B * c.N * c.Sk
+        fwd_bytes = (2 * rows_q + 2 * rows_k) * c.D * esz + 4 * rows_q
+        bwd_bytes = (4 * rows_q + 4 * rows_k) * c.D * esz + 4 * rows_q
+        line = {"metric": METRIC, "config": c.name, "label": label,
+                "dtype": {torch.bfloat16: "bf16", torch.float32: "f32"}[q.dtype],
+                "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4),
+                "fwd_tflops": round(nominal / (f_ms * 1e-3) / 1e12, 2),
+                "fwd_tflops_allowed_pairs": round(allowed / (f_ms * 1e-3) / 1e12, 2),
+                "bwd_tflops": round(2.5 * nominal / (b_ms * 1e-3) / 1e12, 2),
+                "bwd_tflops_allowed_pairs": round(2.5 * allowed / (b_ms * 1e-3) / 1e12, 2),
+                "fwd_frac_of_peak": round(nominal / (f_ms * 1e-3) / 1e12 / peak, 4),
+                "fwd_gbs": round(fwd_bytes / (f_ms * 1e-3) / 1e9, 1),
+                "bwd_gbs": round(bwd_bytes / (b_ms * 1e-3) / 1e9, 1),
+                "peak": peak, "peak_kind": f"{pk_kind} bf16_tflops (burst)",
+                "l2_flushed_between_reps": do_flush, "timing": "median of 30 after 10 warm-ups"}
+        print(json.dumps(line), flush=True)
+        del dev, out, lse, ws
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -497,11 +593,16 @@ def main():
     ap.add_argument("--cpu-seq", type=int, default=512,
                     help="token prefix of the oracle's bounded sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--configs", action="store_true",
+                    help="instead of the main line, time every workload of the "
+                         "source pages (one JSON line each)")
     args = ap.parse_args()
     if args.impl == "ours":
         args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     if args.impl == "reference":
         run_reference(args)
+    elif args.configs:
+        run_configs(args)
     else:
         run_ours(args)
 
