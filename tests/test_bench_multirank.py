@@ -1,4 +1,4 @@
-"""The bench's multi-rank plumbing on CPU: two gloo ranks stand in for two
+"""The bench's host-side logic on CPU.  Multi-rank plumbing: two gloo ranks stand in for two
 GPUs (one process per GPU under torchrun).  Checked: every rank joins the
 same collectives, the reported time is the maximum over ranks, the
 whole-job value counts every rank's work (weak scaling), and the reference
@@ -64,3 +64,27 @@ def test_single_rank_value_is_per_gpu_work():
     import bench
     assert bench.max_over_ranks(4.2, 1) == 4.2
     assert bench.whole_job_value(2e12, 1, 10.0) == pytest.approx(200.0)
+
+
+def test_allowed_pairs_matches_brute_force():
+    # the per-workload sweep's "allowed pairs" count, against a direct loop
+    sys.path.insert(0, ROOT)
+    import bench
+    from attention_fwd_bwd_02_b200 import inputs as I
+    cases = [I.make_case("ap_mod", 2, 3, 12, 12, 64, modality=(4, 8)),
+             I.make_case("ap_pad", 3, 2, 5, 9, 64, kv_len_range=(0, 9)),
+             I.make_case("ap_causal", 1, 2, 7, 7, 64, causal=True),
+             I.make_case("ap_diag", 1, 1, 6, 6, 64, modality=(2, 4),
+                         allow=((0, 1), (1, 0)), allow_diag=True)]
+    for c in cases:
+        n = 0
+        for b in range(c.B):
+            nk = c.Sk if c.kv_len is None else int(c.kv_len[b])
+            for i in range(c.Sq):
+                for j in range(c.Sk):
+                    ok = j < nk and (not c.causal or j <= i)
+                    if c.modality_ids is not None:
+                        a, e = int(c.modality_ids[b, i]) & 1, int(c.modality_ids[b, j]) & 1
+                        ok = ok and (bool(c.allow[a][e]) or (c.allow_diag and i == j))
+                    n += ok
+        assert bench._allowed_pairs(c) == n * c.N, c.name
