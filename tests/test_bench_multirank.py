@@ -1,8 +1,10 @@
-"""The bench's host-side logic on CPU.  Multi-rank plumbing: two gloo ranks stand in for two
-GPUs (one process per GPU under torchrun).  Checked: every rank joins the
-same collectives, the reported time is the maximum over ranks, the
-whole-job value counts every rank's work (weak scaling), and the reference
-arm prints only on rank 0."""
+"""The bench's host-side logic on CPU.
+
+Multi-rank plumbing: two gloo ranks stand in for two GPUs (one process per
+GPU under torchrun).  Checked: every rank joins the same collectives, the
+reported time is the maximum over ranks, the whole-job value counts every
+rank's work (weak scaling), and the reference arm prints only on rank 0.
+Also the per-workload sweep's count of visible (query, key) pairs."""
 import contextlib
 import io
 import os
