@@ -43,6 +43,15 @@ def test_bf16_causal_alibi(D, S):
     check_bwd(c)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("S", [128, 300])
+def test_bf16_causal_no_alibi(D, S):
+    # The causal rule alone: full tiles take the unmasked branch of the
+    # softmax, the diagonal tiles the masked one, with no bias term.
+    c = I.make_case(f"bwd_c_D{D}_S{S}", 2, 3, S, S, D, seed=38, causal=True)
+    check_bwd(c)
+
+
 def test_bf16_padding_with_empty_batch():
     c = I.make_case("bwd_pad", 4, 2, 32, 300, 64, seed=33, kv_len_range=(0, 300))
     c.kv_len[0] = 0
@@ -101,6 +110,13 @@ def test_empty_query_and_key_sets():
 
 
 # ------------------------------------------------------------ full workloads
+
+def test_config2_causal_bwd_full_size_sampled():
+    # The causal B=4 N=32 S=2048 D=128 workload, no bias, exactly as timed.
+    c = I.config2(with_dout=True)
+    heads = [(0, 0), (1, 17), (3, 31)]
+    check_bwd(c, heads=heads)
+
 
 @pytest.mark.parametrize("S,D", I.CONFIG5_SWEEP)
 def test_config5_fwd_bwd_full_size_sampled(S, D):

@@ -27,6 +27,10 @@ MUTATIONS = {
                 "ds[(int64_t)i * Sk + j] = pij * (dl - ds[(int64_t)i * Sk + j]);"),
     "modality_transposed": ("else if (a == 0 && c == 1) ok = m->allow01;",
                             "else if (a == 0 && c == 1) ok = m->allow10;"),
+    "diagonal_ignored": ("if (m->allow_diag && i == j) ok = 1;",
+                         "if (m->allow_diag && i == j) ok = ok;"),
+    "diagonal_on_ids": ("if (m->allow_diag && i == j) ok = 1;",
+                        "if (m->allow_diag && a == c) ok = 1;"),
     "dq_uses_q": ("acc += ds[(int64_t)i * Sk + j] * kh[(int64_t)j * D + d];",
                   "acc += ds[(int64_t)i * Sk + j] * qh[(int64_t)j * D + d];"),
 }
@@ -37,6 +41,8 @@ CHECKS = [
     pins.test_alibi_q0_closed_form,
     lambda: pins.test_q_zero_gives_mean_of_allowed_v("padding"),
     lambda: pins.test_q_zero_gives_mean_of_allowed_v("modality"),
+    lambda: pins.test_hand_cross_modal_diagonal("page_rule"),
+    lambda: pins.test_hand_cross_modal_diagonal("image_only_with_diag"),
     lambda: pins.test_matches_torch_sdpa_fwd_bwd("causal", (13, 13)),
     lambda: pins.test_matches_torch_sdpa_fwd_bwd("padding", (7, 19)),
     lambda: pins.test_bwd_finite_differences("none", True),

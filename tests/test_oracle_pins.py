@@ -93,9 +93,41 @@ def test_alibi_q0_closed_form():
                 assert abs(out[0, 0, i, 0] - mean_j) < 1e-12
 
 
+def _expr(x):
+    """A fixture value written as an exact expression: numbers, fractions,
+    natural logs ln(.) and -inf."""
+    if x == "-inf":
+        return -math.inf
+    return float(eval(x, {"__builtins__": {}}, {"ln": math.log}))
+
+
+@pytest.mark.parametrize("case", ["page_rule", "workload_rule", "image_only_with_diag",
+                                  "image_only_no_diag"])
+def test_hand_cross_modal_diagonal(case):
+    g = json.load(open(os.path.join(GOLD, "hand_cross_modal_diag.json")))
+    S = g["shape"]["S"]
+    vec = lambda key: np.array([_expr(x) for x in g[key]]).reshape(1, 1, S, 1)
+    q, k, v, do = vec("q"), vec("k"), vec("v"), vec("dout")
+    ids = np.array([g["ids"]], dtype=np.int32)
+    c = g["cases"][case]
+    kw = dict(modality_ids=ids, allow=tuple(map(tuple, c["allow"])), allow_diag=c["allow_diag"])
+    out, lse = oracle.fwd(q, k, v, g["scale"], **kw)
+    np.testing.assert_allclose(out.reshape(-1), [_expr(x) for x in c["out"]], rtol=0, atol=1e-14)
+    exp_lse = np.array([_expr(x) for x in c["lse"]])
+    assert np.array_equal(np.isneginf(lse.reshape(-1)), np.isneginf(exp_lse))
+    fin = np.isfinite(exp_lse)
+    np.testing.assert_allclose(lse.reshape(-1)[fin], exp_lse[fin], rtol=0, atol=1e-14)
+    if "dq" in c:
+        dq, dk, dv = oracle.bwd(q, k, v, do, g["scale"], **kw)
+        for name, got in (("dq", dq), ("dk", dk), ("dv", dv)):
+            np.testing.assert_allclose(got.reshape(-1), [_expr(x) for x in c[name]],
+                                       rtol=0, atol=1e-14, err_msg=name)
+
+
 # ---------------------------------------------------------------- closed forms
 
-MASK_MODES = ["none", "causal", "padding", "bool", "modality", "causal+padding"]
+MASK_MODES = ["none", "causal", "padding", "bool", "modality", "modality_page",
+              "causal+padding"]
 
 
 def _mask_kwargs(mode, B, N, Sq, Sk, seed=0):
@@ -113,6 +145,16 @@ def _mask_kwargs(mode, B, N, Sq, Sk, seed=0):
         ids[:, Sk // 3:] = 1
         kw["modality_ids"] = ids
         kw["allow"] = ((1, 1), (0, 1))
+    if mode == "modality_page":
+        # The multimodal page's own cross-modal rule (layer 2,
+        # create_cross_modal_mask): a token attends the other modality and
+        # itself, never another token of its own modality.
+        assert Sq == Sk
+        ids = np.zeros((B, Sk), dtype=np.int32)
+        ids[:, Sk // 3:] = 1
+        kw["modality_ids"] = ids
+        kw["allow"] = ((0, 1), (1, 0))
+        kw["allow_diag"] = True
     return kw
 
 
@@ -132,6 +174,8 @@ def _allowed_dense(mode, B, N, Sq, Sk, kw):
         ids = torch.as_tensor(kw["modality_ids"]).long()
         allow = torch.as_tensor(kw["allow"]).bool()
         pair = allow[ids[:, :, None], ids[:, None, :]]   # [B, Sq, Sk]
+        if kw.get("allow_diag"):
+            pair |= torch.eye(Sq, Sk, dtype=torch.bool)[None]
         a &= pair[:, None]
     return a
 
@@ -194,7 +238,7 @@ def test_causal_row0_and_sk1():
 @pytest.mark.parametrize("sq_sk", [(13, 13), (7, 19)])
 def test_matches_torch_sdpa_fwd_bwd(mode, sq_sk):
     Sq, Sk = sq_sk
-    if mode == "modality" and Sq != Sk:
+    if mode.startswith("modality") and Sq != Sk:
         pytest.skip("modality rule is self-attention only")
     B, N, D = 2, 3, 8
     scale = 0.37
@@ -314,7 +358,8 @@ def _loss(q, k, v, do, scale, kw):
     return float((out * do).sum())
 
 
-@pytest.mark.parametrize("mode", ["none", "causal", "padding", "bool", "modality"])
+@pytest.mark.parametrize("mode", ["none", "causal", "padding", "bool", "modality",
+                                  "modality_page"])
 @pytest.mark.parametrize("alibi", [False, True])
 def test_bwd_finite_differences(mode, alibi):
     B, N, S, D = 1, 2, 5, 3
