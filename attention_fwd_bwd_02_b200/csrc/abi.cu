@@ -9,13 +9,16 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/fa.h"
 #include "../../include/fa_testing.h"
 #include "fa_common.cuh"
 #include "launch.h"
 
 namespace fa {
-// Device status word: kernels OR bit 0 into it when a bounded wait gives up.
+// Device status word: kernels OR bit 0 into it when a bounded wait gives up,
+// bit 1 when a persistent kernel lost its work counter to a later launch.
 __device__ unsigned int g_fa_status = 0;
 }  // namespace fa
 
@@ -119,12 +122,17 @@ fa_status make_problem(const fa_shape* s, const fa_pse* pse, const fa_mask* m,
   return FA_OK;
 }
 
-// Device address of g_fa_status on the current device (looked up once per
-// device; the symbol lives in every device's copy of the module).
+// Device address of g_fa_status on the current device, looked up once per
+// device (the symbol lives in every device's copy of the module) under a
+// lock, so that threads making their first call at once agree.  The cached
+// address assumes the module stays loaded: cudaDeviceReset is not supported
+// while the library is in use.
 unsigned int* status_word() {
+  static std::mutex mu;
   static unsigned int* addr[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
   if (!addr[dev]) {
     void* a = nullptr;
     if (cudaGetSymbolAddress(&a, fa::g_fa_status) != cudaSuccess) return nullptr;
@@ -162,6 +170,7 @@ const char* fa_status_string(fa_status status) {
     case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
     case FA_ERR_CUDA: return "FA_ERR_CUDA";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    case FA_ERR_CONCURRENT: return "FA_ERR_CONCURRENT";
   }
   return "FA_ERR_UNKNOWN";
 }
@@ -326,8 +335,12 @@ fa_status fa_sync_status(void* stream) {
   if (word != 0) {
     e = cudaMemcpyToSymbol(fa::g_fa_status, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_status(e);
+    // A kernel that gave up may have left its work counter mid-count.
+    e = fa::reset_work_counters();
+    if (e != cudaSuccess) return cuda_status(e);
   }
-  return word ? FA_ERR_TIMEOUT : FA_OK;
+  if (word & 1u) return FA_ERR_TIMEOUT;
+  return word ? FA_ERR_CONCURRENT : FA_OK;
 }
 
 }  // extern "C"

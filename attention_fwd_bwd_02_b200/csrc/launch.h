@@ -26,9 +26,12 @@ cudaError_t launch_bwd_sm100(const Problem& p, const void* q, const void* k,
                              const float* delta, float* dq_acc, void* dk,
                              void* dv, cudaStream_t st);
 
-// Dynamic scheduler of the persistent kernels (sched.cu): a cleared-per-
-// launch work counter (the caller clears it on its stream) and the SM count.
+// Dynamic scheduler of the persistent kernels (sched.cu, sched.cuh): the
+// work counter slot of one launch (null if the device could not be
+// queried), the clearing of every slot after a kernel gave up a wait, and
+// the SM count.
 unsigned int* work_counter();
+cudaError_t reset_work_counters();
 int sm_count();
 
 // Helpers (aux.cu), for tensors of element type `elem`.

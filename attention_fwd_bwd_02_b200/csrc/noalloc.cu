@@ -23,7 +23,9 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_NOALLOC_SCRA
 
 // Device address of g_noalloc_scratch on the current device.  In host code
 // the array's name only stands in for the symbol, so the address is looked
-// up once per device, with that device current.
+// up once per device, with that device current.  The cached address assumes
+// the module stays loaded (cudaDeviceReset is not supported while the
+// library is in use).
 cudaError_t scratch_address(void** out) {
   static std::mutex mu;
   static void* addr[64] = {};
@@ -52,6 +54,12 @@ extern "C" fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q,
                                     float keep_prob, void* dq, void* dk,
                                     void* dv, void* stream) {
   if (!shape) return FA_ERR_INVALID_ARG;
+  if (shape->B == 0 || shape->N == 0 || shape->Sq == 0 || shape->Sk == 0) {
+    // No (query, key) pair: fa_bwd needs no workspace for this shape, so
+    // its result and status come without touching the scratch array.
+    return fa_bwd(shape, q, k, v, out, dout, lse, pse, mask, scale, keep_prob,
+                  dq, dk, dv, nullptr, 0, stream);
+  }
   const size_t need = fa_bwd_workspace_size(shape);
   if (need == 0 && shape->B > 0 && shape->N > 0 && shape->Sq > 0) {
     // An invalid shape: fa_bwd reports the precise status without touching

@@ -24,7 +24,8 @@ LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "fa.h")
 TESTING_HEADER = os.path.join(os.path.dirname(_HERE), "include", "fa_testing.h")
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+(FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT,
+ FA_ERR_CONCURRENT) = range(6)
 FA_LAYOUT_BNSD, FA_LAYOUT_BSH = 0, 1
 FA_F32, FA_BF16, FA_F16 = 0, 1, 2
 FA_MASK_CAUSAL, FA_MASK_KV_PADDING, FA_MASK_BOOL, FA_MASK_MODALITY = 1, 2, 4, 8
@@ -67,7 +68,7 @@ _lib = None
 
 def _status_name(s):
     names = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED",
-             3: "FA_ERR_CUDA", 4: "FA_ERR_TIMEOUT"}
+             3: "FA_ERR_CUDA", 4: "FA_ERR_TIMEOUT", 5: "FA_ERR_CONCURRENT"}
     return names.get(int(s), "FA_ERR_UNKNOWN")
 
 

@@ -17,7 +17,10 @@
  * --------------------------------
  *  - All tensor pointers are DEVICE pointers, allocated and owned by the
  *    caller.  The library never allocates device memory and keeps no state
- *    between calls, except one device-side status word (fa_sync_status).
+ *    between calls, except one device-side status word (fa_sync_status)
+ *    and the persistent forward's work counters.  Device addresses of these
+ *    are looked up once per device, so cudaDeviceReset is not supported
+ *    while the library is in use.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream).  Every call that launches work is asynchronous on that stream.
  *  - Argument errors are detected on the host before anything is launched
@@ -51,7 +54,10 @@ typedef enum {
   FA_ERR_INVALID_ARG = 1,  /* malformed argument (null, shape, stride)      */
   FA_ERR_UNSUPPORTED = 2,  /* well-formed but not implemented (keep_prob<1) */
   FA_ERR_CUDA = 3,         /* a CUDA runtime call or launch failed          */
-  FA_ERR_TIMEOUT = 4       /* a kernel's bounded wait gave up               */
+  FA_ERR_TIMEOUT = 4,      /* a kernel's bounded wait gave up               */
+  FA_ERR_CONCURRENT = 5    /* more forward calls ran on one GPU at the same
+                              time than the library has work counters (64):
+                              the results of the calls involved are invalid */
 } fa_status;
 
 typedef enum { FA_LAYOUT_BNSD = 0, FA_LAYOUT_BSH = 1 } fa_layout;
@@ -155,6 +161,10 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
  *     returns FA_ERR_UNSUPPORTED without launching anything.
  *   - The first call on a device looks up the array's device address (with
  *     that device current); make that first call before any stream capture.
+ *     The address is kept for the life of the process, so cudaDeviceReset
+ *     is not supported while the library is in use.
+ *   - Shapes with no (query, key) pair (B, N, Sq or Sk equal to 0) go to
+ *     fa_bwd directly and never touch the array.
  *   - All calls share the one array: calls that overlap on the GPU (other
  *     streams, other host threads) race on it and give wrong gradients.
  *     Calls on one stream, or otherwise ordered, are safe; the array keeps
@@ -188,6 +198,8 @@ fa_status fa_build_modality_mask(int B, int S, const int32_t* modality_ids,
 
 /* Synchronises `stream`, then returns and clears the device status word:
  * FA_ERR_TIMEOUT if a kernel gave up a bounded wait since the last call,
+ * FA_ERR_CONCURRENT if a forward found its work counter shared with
+ * another call (only possible with more than 64 forwards running at once),
  * FA_ERR_CUDA if the stream reported an error, else FA_OK. */
 fa_status fa_sync_status(void* stream);
 

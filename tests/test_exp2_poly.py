@@ -13,7 +13,8 @@ SRC = os.path.join(os.path.dirname(exp2_fit.__file__), "csrc", "fwd_sm100.cu")
 
 def _kernel_coeffs():
     src = open(SRC).read()
-    body = src[src.index("exp2_fma_x2("):src.index("constexpr uint32_t kSoftExpPairs")]
+    start = src.index("exp2_fma_x2(")
+    body = src[start:src.index("\n}\n", start)]
     vals = [float(v) for v in re.findall(r"f2_pack\(([0-9.]+)f, \1f\)", body)]
     vals = [v for v in vals if v < 2.0]  # drop the rounding constant
     # order in the source: c3, c2, c1, c0

@@ -27,18 +27,36 @@ def _cuda():
 
 @pytest.mark.parametrize("D", [64, 128])
 def test_noalloc_matches_workspace_backward(D):
-    c = I.make_case(f"noalloc_D{D}", 2, 4, 300, 300, D, seed=41, causal=True, alibi=True)
-    dev = P.to_dev(c)
-    kw = dict(pse=dev["slopes"], scale=c.scale, causal=True)
-    out, lse = fa.fwd(dev["q"], dev["k"], dev["v"], c.N, "BNSD", **kw)
-    ref = fa.bwd(dev["q"], dev["k"], dev["v"], out, dev["dout"], lse, c.N, "BNSD", **kw)
-    for call in range(2):
+    # Two calls in a row on different inputs and shapes: the second call
+    # finds the first call's data in the shared scratch array, and its
+    # result must match fa_bwd (caller workspace) on its own inputs.
+    cases = [I.make_case(f"noalloc_D{D}_a", 2, 4, 300, 300, D, seed=41, causal=True, alibi=True),
+             I.make_case(f"noalloc_D{D}_b", 1, 3, 200, 200, D, seed=42, causal=True)]
+    for call, c in enumerate(cases):
+        dev = P.to_dev(c)
+        kw = dict(pse=dev["slopes"], scale=c.scale, causal=True)
+        out, lse = fa.fwd(dev["q"], dev["k"], dev["v"], c.N, "BNSD", **kw)
+        ref = fa.bwd(dev["q"], dev["k"], dev["v"], out, dev["dout"], lse, c.N, "BNSD", **kw)
+        grads = tuple(torch.full_like(t, float("nan")) for t in (dev["q"], dev["k"], dev["v"]))
+        torch.cuda.synchronize()
+        before = torch.cuda.memory_allocated()
+        torch.cuda.reset_peak_memory_stats()
         got = fa.bwd_noalloc(dev["q"], dev["k"], dev["v"], out, dev["dout"], lse, c.N,
-                             "BNSD", **kw)
+                             "BNSD", dq=grads[0], dk=grads[1], dv=grads[2], **kw)
         fa.sync_status()
+        # Nothing was allocated through the caller's allocator, even for a
+        # moment (the peak stays at the level before the call).
+        assert torch.cuda.max_memory_allocated() <= before, "the call allocated device memory"
+        assert all(g is t for g, t in zip(got, grads))
         for name, g, r in zip(("dq", "dk", "dv"), got, ref):
             P.assert_close(g.double().cpu().numpy(), r.double().cpu().numpy(), c.dtype,
                            f"call {call} {name}")
+
+
+def test_noalloc_empty_shape_is_a_no_op():
+    s = fa.FaShape(0, 4, 128, 128, 64, fa.FA_LAYOUT_BNSD, fa.FA_BF16)
+    assert fa.lib().fa_bwd_noalloc(s, None, None, None, None, None, None, None, None,
+                                   0.1, 1.0, None, None, None, None) == fa.FA_OK
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
