@@ -6,29 +6,29 @@
 // sec. 2 formula; sec. 3.2 parameters), tile by tile with an online softmax
 // so the score matrix never leaves the SM.
 //
-// Persistent kernel: one CTA per SM.  A work item is two 128-row query tiles
-// (256 rows) of one (b, h); the CTA walks the 128-key tiles that the mask
-// leaves visible.  The two query tiles ping-pong on the tensor core: while
-// the softmax warps of one tile turn S into P, the tensor core runs P V and
-// the next Q K^T of the other.  The MMA stream runs on across work items
-// (the last P V of an item is issued together with the first Q K^T of the
-// next), so the ping-pong does not stop at item boundaries.
-// Warp roles (16 warps):
+// Persistent kernel: one CTA per SM walks a static list of work items.  A
+// work item is two 128-row query tiles (256 rows) of one (b, h); the CTA walks
+// the key tiles (128 keys each) that the mask leaves visible.  The two query
+// tiles ping-pong on the tensor core: while the softmax warps of one tile
+// turn S into P, the tensor core runs P V and Q K^T of the other.  Items are
+// ordered longest first under the causal mask and dealt round-robin, so the
+// CTAs finish together; the loads of the next item overlap the tail of the
+// current one.
+// Warp roles:
 //   warps 0-3 / 4-7  softmax of query tile 0 / 1: thread t owns query row t.
 //              Reads S from TMEM, applies scale / ALiBi / mask, updates the
-//              running max and sum, writes P (operand type) back into TMEM
-//              over S, rescales O in TMEM when the running max grew by more
-//              than 2^8, and writes the LSE at the end of an item.
-//   warps 8-11 epilogue of both tiles: O / l from TMEM to global memory.
-//   warp 12    TMA producer: Q tiles per item, then K_j and V_j through one
-//              ring of stages.
-//   warp 13    MMA issuer and TMEM owner:
+//              running max and sum, writes P (operand type) back into TMEM over S,
+//              rescales O in TMEM when the running max grew by more than
+//              2^8, and at the end of an item writes O / l and the LSE.
+//   warp 8     TMA producer: both Q tiles per item, then K_j and V_j through
+//              two separate rings of stages.
+//   warp 9     MMA issuer (one elected lane) and TMEM owner:
 //              S_t = Q_t K_j^T (SS form), O_t += P_t V_j (P from TMEM, TS form).
-//   warp 14    scheduler: claims work items ahead of the other roles.
-//   warp 15    idle.
-// TMEM columns: S/P of tile t at 128 t; O_t at 256 + D t.  Shared memory
-// holds every operand as 128-byte-swizzled 64-column boxes, the canonical
-// layout of both TMA and tcgen05 descriptors.
+//   warps 10-11 idle (they complete the third warpgroup, which gives its
+//              registers to the softmax warpgroups).
+// TMEM columns: S/P of tile 0 at 0, of tile 1 at 128; O_0 at 256, O_1 at
+// 256 + D.  Shared memory holds every operand as 128-byte-swizzled 64-column
+// boxes, the canonical layout of both TMA and tcgen05 descriptors.
 //
 // The Ascend design on the source pages splits the work between a matrix
 // unit and vector units (Cube/Vector overlap); here the same overlap comes
@@ -36,8 +36,6 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
-
-#include <atomic>
 
 #include "fa_common.cuh"
 #include "launch.h"
@@ -54,34 +52,19 @@ constexpr int kTiles = 2;             // query tiles per work item
 constexpr int kRows = kBM * kTiles;   // query rows per work item
 constexpr int kBN = 128;              // keys per tile
 constexpr int kBoxBytes = 128 * 128;  // one 128-row x 64-col 16-bit box
-constexpr int kThreads = 512;         // 4 warpgroups
+constexpr int kThreads = 384;         // 3 warpgroups
 constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only if max grows > 2^8
-constexpr int kSchedRing = 2;         // work items in flight between roles
-constexpr int kStepRing = 16;         // MMA step commands in flight
-// The two softmax warps of a sub-partition (tile 0 and tile 1 of the same
-// TMEM lane quarter) take turns for the exponential phase of a step:
-// 0 = no turns, 1 = the turn covers the S load, row max and exponentials,
-// 2 = row max and exponentials only.
-#ifndef FA_SOFTMAX_TURNS
-#define FA_SOFTMAX_TURNS 0
-#endif
-constexpr int kSoftmaxTurns = FA_SOFTMAX_TURNS;
-constexpr int kWarpEpi = 8, kWarpLoad = 12, kWarpMma = 13, kWarpSched = 14;
-// Readers of a scheduled item id (one arrival per warp): the producer and
-// the 8 softmax warps.  The MMA warp takes its steps from the producer and
-// the epilogue warps learn the items from the softmax warps (the per-tile
-// records below).
+constexpr int kSchedRing = 4;         // work items in flight between roles
+// Consumers of a scheduled item id: the MMA warp and the 8 softmax warps.
 constexpr int kSchedConsumers = 9;
-// Register split.  Launch: 512 threads x 128 = 65536 registers.  After the
-// split: 2 softmax warpgroups x 128 x 208 + epilogue warpgroup x 128 x 40 +
-// control warpgroup x 128 x 56 = 53248 + 5120 + 7168 = 65536.
-constexpr uint32_t kRegsLaunch = 128;
+// Register split.  Launch: 384 threads x 168 = 64512 registers.  After the
+// split: 2 softmax warpgroups x 128 x 208 + 1 control warpgroup x 128 x 88
+// = 53248 + 11264 = 64512, the same total.
+constexpr uint32_t kRegsLaunch = 168;
 constexpr uint32_t kRegsSoftmax = 208;
-constexpr uint32_t kRegsEpi = 40;
-constexpr uint32_t kRegsControl = 56;
-static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsEpi + 128 * kRegsControl <=
-                  kThreads * kRegsLaunch,
+constexpr uint32_t kRegsControl = 88;
+static_assert(2 * 128 * kRegsSoftmax + 128 * kRegsControl <= kThreads * kRegsLaunch,
               "register split exceeds the launch allocation");
 
 // 2^x on the FMA pipe, for the share of the exponentials that the MUFU unit
@@ -95,7 +78,7 @@ __device__ __forceinline__ void exp2_fma_x2(float a0, float a1, float& p0, float
   const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
   const uint64_t neg_magic = f2_pack(-12582912.0f, -12582912.0f);
   const uint64_t minus_one = f2_pack(-1.0f, -1.0f);
-  const uint64_t x2 = f2_pack(fmaxf(a0, -127.0f), fmaxf(a1, -127.0f));
+  const uint64_t x2 = f2_pack(a0, a1);
   const uint64_t y2 = fadd2(x2, magic);         // j in the low mantissa bits
   const uint64_t j2 = fadd2(y2, neg_magic);     // rint(x), exact
   const uint64_t f2 = ffma2(j2, minus_one, x2);  // x - j, exact
@@ -112,48 +95,38 @@ __device__ __forceinline__ void exp2_fma_x2(float a0, float a1, float& p0, float
   p1 = a1 < -126.0f ? 0.0f : p1;
 }
 
+// Pairs (of the 16 in a 32-column chunk) whose exponentials use exp2_fma_x2.
+// Measured on B200 with the current softmax schedule, moving half of them
+// to the FMA pipe (0xAAAA) was slower than the MUFU alone (564 vs 713
+// TFLOP/s, causal S=2048 D=128): the step is issue-bound, not MUFU-bound, so
+// every exponential stays on the MUFU for now.
+constexpr uint32_t kSoftExpPairs = 0x0000u;
+
 template <int D>
 struct FwdCfg {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // 128 rows x D
-  // One ring of stages holds K_j and V_j alternately (the producer fills
-  // K_0, V_0, K_1, V_1, ...).
-  static constexpr int kStages = (D == 128) ? 5 : 12;
+  static constexpr int kKStages = (D == 128) ? 2 : 3;
+  static constexpr int kVStages = (D == 128) ? 2 : 3;
   static constexpr int kColO = 256;  // O_t at kColO + t * D
   static constexpr int kSmemQ = 0;
-  static constexpr int kSmemRing = kTiles * kTileBytes;
-  static constexpr int kSmemBar = kSmemRing + kStages * kTileBytes;
-  // q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2],
-  // o_final[2], o_empty[2], stats_full[2], stats_empty[2], drain,
-  // sched_full[R], sched_empty[R], step_full[T], step_empty[T]
-  static constexpr int kNumBars = 4 + 2 * kStages + 12 + 1 + 2 * kSchedRing + 2 * kStepRing;
-  static constexpr int bQFull = 0, bQEmpty = 2, bKvFull = 4, bKvEmpty = bKvFull + kStages;
-  static constexpr int bSFull = bKvEmpty + kStages, bPFull = bSFull + 2;
-  static constexpr int bOFinal = bPFull + 2, bOEmpty = bOFinal + 2;
-  static constexpr int bStatsFull = bOEmpty + 2, bStatsEmpty = bStatsFull + 2;
-  static constexpr int bDrain = bStatsEmpty + 2;
+  static constexpr int kSmemK = kTiles * kTileBytes;
+  static constexpr int kSmemV = kSmemK + kKStages * kTileBytes;
+  static constexpr int kSmemBar = kSmemV + kVStages * kTileBytes;
+  // q_full[2], q_empty[2], k_full[SK], k_empty[SK], v_full[SV], v_empty[SV],
+  // s_full[2], p_full[2], o_final[2], o_empty[2], drain, sched_full[R],
+  // sched_empty[R]
+  static constexpr int kNumBars = 4 + 2 * kKStages + 2 * kVStages + 8 + 1 + 2 * kSchedRing;
+  // barrier indices
+  static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = bKFull + kKStages;
+  static constexpr int bVFull = bKEmpty + kKStages, bVEmpty = bVFull + kVStages;
+  static constexpr int bSFull = bVEmpty + kVStages, bPFull = bSFull + 2;
+  static constexpr int bOFinal = bPFull + 2, bOEmpty = bOFinal + 2, bDrain = bOEmpty + 2;
   static constexpr int bSchedFull = bDrain + 1, bSchedEmpty = bSchedFull + kSchedRing;
-  static constexpr int bStepFull = bSchedEmpty + kSchedRing, bStepEmpty = bStepFull + kStepRing;
-  static constexpr int kSmemMisc = kSmemBar + kNumBars * 8;   // tmem addr, abort flags
+  static constexpr int kSmemMisc = kSmemBar + kNumBars * 8;  // tmem addr, abort
   static constexpr int kSmemSched = kSmemMisc + 16;           // int[kSchedRing]
-  // Per query tile, the record of its last finished item: a header
-  // {b, h, q0, flags} and 1 / l of each row.
-  static constexpr int kSmemSteps = kSmemSched + 4 * kSchedRing;  // uint32[kStepRing]
-  static constexpr int kSmemLock = kSmemSteps + 4 * kStepRing;  // uint32[4]
-  static constexpr int kSmemRec = kSmemLock + 16;
-  static constexpr int kRecBytes = 16 + 4 * kBM;
-  static constexpr int kSmemBytes = kSmemRec + kTiles * kRecBytes + 1024;
-  static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static constexpr int kSmemBytes = kSmemSched + 4 * kSchedRing + 1024;
 };
-
-// A step command from the producer to the MMA warp: one visited key tile
-// (its K and V occupy the next two ring stages).  Bit t: tile t visits it;
-// bit 2 + t: first visit of tile t in its item; bit 4 + t: last visit.
-constexpr uint32_t kStepEnd = 1u << 31;  // no more steps
-
-// Flags of a per-tile item record.
-constexpr uint32_t kRecHaveO = 1u;  // the tile visited key tiles: O_t holds its sum
-constexpr uint32_t kRecDone = 2u;   // no more items for this tile
 
 // One work item: two query tiles of one (b, h).
 struct Item {
@@ -284,104 +257,6 @@ __device__ __forceinline__ int tile_class(const Problem& p, const Item& c, int t
   return cls;
 }
 
-// Warp-collective: whether tile t of the item visits any key tile, and the
-// last key tile it visits (-1 if none).
-__device__ __forceinline__ int last_visited(const Problem& p, const Item& c, int t) {
-  if (!has_rows(c, t)) return -1;
-  for (int kt = c.kt_end - 1; kt >= 0; --kt)
-    if (tile_class(p, c, t, kt, key_tile_ids(p, c, kt)) != 0) return kt;
-  return -1;
-}
-
-// Waits on `bar` until the phase with this parity completes; every lane of
-// the warp calls it, and all lanes agree on the result.
-__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, uint32_t abort_addr) {
-  return __all_sync(~0u, mbar_wait_s(bar, parity, abort_addr));
-}
-
-// Reads item slot n of the schedule ring (warp-collective) and releases it.
-template <class C>
-__device__ __forceinline__ int read_item(uint32_t sb, int n, uint32_t abort_addr, bool& ok) {
-  const int slot = n % kSchedRing;
-  const uint32_t full = sb + uint32_t(C::kSmemBar + 8 * (C::bSchedFull + slot));
-  const uint32_t empty = sb + uint32_t(C::kSmemBar + 8 * (C::bSchedEmpty + slot));
-  if (!warp_wait(full, (n / kSchedRing) & 1, abort_addr)) {
-    ok = false;
-    return -1;
-  }
-  const int w = int(ld_shared_volatile(sb + C::kSmemSched + 4u * slot));
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0) mbar_arrive(empty);
-  return w;
-}
-
-// Softmax warpgroup of tile t: publishes the record of its finished item
-// (or the final "done" record) for the epilogue warps, once they have taken
-// the previous one.  Each of the 128 threads writes its row's 1 / l; row 0
-// writes the header.
-template <class C>
-__device__ __forceinline__ bool publish_record(uint32_t sb, uint32_t rec, int t, int row,
-                                               int& cnt, uint32_t abort_addr, int b, int h,
-                                               int q0, uint32_t flags, float inv) {
-  const uint32_t full = sb + uint32_t(C::kSmemBar + 8 * (C::bStatsFull + t));
-  const uint32_t empty = sb + uint32_t(C::kSmemBar + 8 * (C::bStatsEmpty + t));
-  if (cnt > 0 && !warp_wait(empty, (cnt - 1) & 1, abort_addr)) return false;
-  const uint32_t rt = rec + t * C::kRecBytes;
-  st_shared_u32(rt + 16 + 4 * row, __float_as_uint(inv));
-  if (row == 0) {
-    st_shared_u32(rt + 0, uint32_t(b));
-    st_shared_u32(rt + 4, uint32_t(h));
-    st_shared_u32(rt + 8, uint32_t(q0));
-    st_shared_u32(rt + 12, flags);
-  }
-  mbar_arrive(full);
-  ++cnt;
-  return true;
-}
-
-// Turn-taking between the two softmax warps of one sub-partition: a lock
-// word in shared memory, taken by lane 0 with compare-and-swap (backing off
-// with a short sleep so the holder keeps the issue slots) and released with
-// an exchange.  It orders no data; it only keeps the two warps' MUFU-bound
-// phases from overlapping.  Bounded like every wait: after about a second
-// the waiter gives up the turn-taking (and raises the abort flag).
-__device__ __forceinline__ void turn_acquire(uint32_t lock, uint32_t abort_addr) {
-  if ((threadIdx.x & 31) == 0) {
-    uint32_t it = 0;
-    uint64_t t0 = 0;
-    while (true) {
-      uint32_t old;
-      asm volatile("atom.shared.cas.b32 %0, [%1], 0, 1;" : "=r"(old) : "r"(lock) : "memory");
-      if (old == 0) break;
-      __nanosleep(32);
-      if ((++it & 63u) == 0) {
-        if (ld_shared_volatile(abort_addr)) break;
-        const uint64_t now = globaltimer_ns();
-        if (t0 == 0) t0 = now;
-        else if (now - t0 > 1000000000ull) {
-          st_shared_u32(abort_addr, 1u);
-          break;
-        }
-      }
-    }
-  }
-  __syncwarp();
-}
-__device__ __forceinline__ void turn_release(uint32_t lock) {
-  __syncwarp();
-  if ((threadIdx.x & 31) == 0)
-    asm volatile("atom.shared.exch.b32 _, [%0], 0;" ::"r"(lock) : "memory");
-}
-
-// Loads cols [c0, c0+64) of a 128-column S row block and waits: two x32 loads.
-__device__ __forceinline__ void tmem_ld64_wait(uint32_t taddr, uint32_t (&a)[32],
-                                               uint32_t (&b)[32]) {
-  tmem_ld32(taddr, a);
-  tmem_ld32(taddr + 32, b);
-  tmem_ld_wait(a);
-  tmem_ld_wait(b);
-}
-
 // kF16 selects fp16 operands (Q, K, V, P, out); bf16 otherwise.
 template <int D, bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -391,20 +266,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               uint16_t* __restrict__ out, float* __restrict__ lse, int q_blocks,
               int n_items, int group, unsigned int* __restrict__ sched_ctr) {
   using C = FwdCfg<D>;
-  // Pairs (of the 16 in a 32-column chunk) whose exponentials use the FMA
-  // pipe instead of the MUFU unit.
-  constexpr uint32_t kEmuPairs = (D == 128) ? 0x0000u : 0x1111u;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // 32-bit shared-window addresses: only the base lives in a register.
   const uint32_t sb = smem_u32(smem);
-  const uint32_t sQa = sb + C::kSmemQ, sRa = sb + C::kSmemRing;
+  const uint32_t sQa = sb + C::kSmemQ, sKa = sb + C::kSmemK, sVa = sb + C::kSmemV;
   auto BAR = [sb](int i) -> uint32_t { return sb + uint32_t(C::kSmemBar + 8 * i); };
   const uint32_t tmem_slot = sb + C::kSmemMisc;
   const uint32_t abort_addr = sb + C::kSmemMisc + 4;
   const uint32_t never_abort = sb + C::kSmemMisc + 8;  // stays 0: unbounded-abort drains
-  const uint32_t rec = sb + C::kSmemRec;  // per-tile item records
+  const uint32_t sched_ids = sb + C::kSmemSched;
+  (void)sQa;
 
   const int warp = threadIdx.x >> 5;
   const int tid = threadIdx.x;
@@ -420,28 +293,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(BAR(C::bPFull + t), 128);
       mbar_init(BAR(C::bOFinal + t), 1);
       mbar_init(BAR(C::bOEmpty + t), 128);
-      mbar_init(BAR(C::bStatsFull + t), 128);
-      mbar_init(BAR(C::bStatsEmpty + t), 128);
     }
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(BAR(C::bKvFull + s), 1);
-      mbar_init(BAR(C::bKvEmpty + s), 1);
+    for (int s = 0; s < C::kKStages; ++s) {
+      mbar_init(BAR(C::bKFull + s), 1);
+      mbar_init(BAR(C::bKEmpty + s), 1);
+    }
+    for (int s = 0; s < C::kVStages; ++s) {
+      mbar_init(BAR(C::bVFull + s), 1);
+      mbar_init(BAR(C::bVEmpty + s), 1);
     }
     mbar_init(BAR(C::bDrain), 1);
     for (int s = 0; s < kSchedRing; ++s) {
       mbar_init(BAR(C::bSchedFull + s), 1);
       mbar_init(BAR(C::bSchedEmpty + s), kSchedConsumers);
     }
-    for (int s = 0; s < kStepRing; ++s) {
-      mbar_init(BAR(C::bStepFull + s), 1);
-      mbar_init(BAR(C::bStepEmpty + s), 1);
-    }
     st_shared_u32(abort_addr, 0u);
     st_shared_u32(never_abort, 0u);
-    for (int q = 0; q < 4; ++q) st_shared_u32(sb + C::kSmemLock + 4 * q, 0u);
     fence_barrier_init();
   }
-  if (warp == kWarpMma) {
+  if (warp == 9) {
     tmem_alloc_s(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
@@ -450,26 +320,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = ld_shared_volatile(tmem_slot);
 
-  if (warp >= kWarpLoad) {
+  if (warp >= 8) {
     reg_dealloc<kRegsControl>();
-    if (warp == kWarpSched) {
-      // -------------------------------------------------------- scheduler
-      if (lane == 0) {
-        for (int n = 0;; ++n) {
-          const int slot = n % kSchedRing;
-          if (n >= kSchedRing &&
-              !mbar_wait_s(BAR(C::bSchedEmpty + slot), ((n / kSchedRing) - 1) & 1, abort_addr))
-            break;
-          const unsigned int idx = claim_item(sched_ctr);
-          const int w = idx < unsigned(n_items) ? int(idx) : -1;
-          if (w < 0) finish_claims(sched_ctr, gridDim.x, n_items, p.status);
-          st_shared_u32(sb + C::kSmemSched + 4u * slot, uint32_t(w));
-          mbar_arrive(BAR(C::bSchedFull + slot));
-          if (w < 0) break;
-        }
-      }
-      __syncwarp();
-    } else if (warp == kWarpLoad) {
+    if (warp == 8) {
       // ---------------------------------------------------------- producer
       // The whole warp walks the schedule (mask classification uses warp
       // votes); lane 0 issues the copies.
@@ -478,314 +331,216 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
       }
-      int ring = 0;  // ring slots filled so far
+      int kidx = 0, vidx = 0;
       int q_uses[kTiles] = {0, 0};
-      int nstep = 0;  // step commands sent
       bool ok = true;
-      // Sends one step command to the MMA warp.
-      auto send_step = [&](uint32_t cmd) -> bool {
-        const int e = nstep % kStepRing;
-        if (nstep >= kStepRing &&
-            !warp_wait(BAR(C::bStepEmpty + e), ((nstep / kStepRing) - 1) & 1, abort_addr))
-          return false;
-        if (lane == 0) {
-          st_shared_u32(sb + C::kSmemSteps + 4u * e, cmd);
-          mbar_arrive(BAR(C::bStepFull + e));
-        }
-        ++nstep;
-        return true;
-      };
       for (int n = 0; ok; ++n) {
-        const int w = read_item<C>(sb, n, abort_addr, ok);
+        // Claim the next work item and publish it to the other roles.
+        const int slot = n % kSchedRing;
+        int w = -1;
+        if (lane == 0) {
+          if (n >= kSchedRing &&
+              !mbar_wait_s(BAR(C::bSchedEmpty + slot), ((n / kSchedRing) - 1) & 1, abort_addr)) {
+            ok = false;
+          } else {
+            const unsigned int idx = claim_item(sched_ctr);
+            w = idx < unsigned(n_items) ? int(idx) : -1;
+            if (w < 0) finish_claims(sched_ctr, gridDim.x, n_items, p.status);
+            st_shared_u32(sched_ids + 4u * slot, uint32_t(w));
+            mbar_arrive(BAR(C::bSchedFull + slot));
+          }
+        }
+        ok = __shfl_sync(~0u, ok, 0);
+        w = __shfl_sync(~0u, w, 0);
         if (!ok || w < 0) break;
         Item c = make_item(p, w, q_blocks, group, causal);
         item_query_ids(p, c);
         const int col0 = bsh ? c.h * D : 0;
         const int z = bsh ? c.b : c.b * p.N + c.h;
-        const int last0 = last_visited(p, c, 0), last1 = last_visited(p, c, 1);
 #pragma unroll
         for (int t = 0; t < kTiles; ++t) {
-          if ((t ? last1 : last0) < 0) continue;  // no Q K^T for this tile
-          if (q_uses[t] > 0 && !warp_wait(BAR(C::bQEmpty + t), (q_uses[t] - 1) & 1, abort_addr)) {
-            ok = false;
-            break;
+          if (!has_rows(c, t)) continue;
+          if (q_uses[t] > 0) {
+            bool got = true;
+            if (lane == 0) got = mbar_wait_s(BAR(C::bQEmpty + t), (q_uses[t] - 1) & 1, abort_addr);
+            if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
           }
           if (lane == 0 && !(p.debug_flags & kDebugWithholdQ)) {
             mbar_arrive_expect_tx(BAR(C::bQFull + t), C::kTileBytes);
             for (int x = 0; x < C::kBoxes; ++x)
               tma_load_3d_s(sQa + t * C::kTileBytes + x * kBoxBytes, &tm_q, BAR(C::bQFull + t),
-                            col0 + 64 * x, c.q0[t], z);
+                          col0 + 64 * x, c.q0[t], z);
           }
           ++q_uses[t];
         }
-        bool first0 = true, first1 = true;
         for (int kt = 0; ok && kt < c.kt_end; ++kt) {
           const uint32_t kid = key_tile_ids(p, c, kt);
-          const bool v0 = tile_class(p, c, 0, kt, kid) != 0;
-          const bool v1 = tile_class(p, c, 1, kt, kid) != 0;
-          if (!v0 && !v1) continue;
-          const uint32_t cmd = (v0 ? 1u : 0u) | (v1 ? 2u : 0u) | ((v0 && first0) ? 4u : 0u) |
-                               ((v1 && first1) ? 8u : 0u) | (kt == last0 ? 16u : 0u) |
-                               (kt == last1 ? 32u : 0u);
-          first0 &= !v0;
-          first1 &= !v1;
-          if (!send_step(cmd)) { ok = false; break; }
-#pragma unroll
-          for (int which = 0; which < 2; ++which) {  // K_kt, then V_kt
-            const int s = ring % C::kStages;
-            if (ring >= C::kStages &&
-                !warp_wait(BAR(C::bKvEmpty + s), ((ring / C::kStages) - 1) & 1, abort_addr)) {
-              ok = false;
-              break;
-            }
-            if (lane == 0) {
-              mbar_arrive_expect_tx(BAR(C::bKvFull + s), C::kTileBytes);
-              for (int x = 0; x < C::kBoxes; ++x)
-                tma_load_3d_s(sRa + s * C::kTileBytes + x * kBoxBytes, which ? &tm_v : &tm_k,
-                              BAR(C::bKvFull + s), col0 + 64 * x, kt * kBN, z);
-            }
-            ++ring;
+          if (tile_class(p, c, 0, kt, kid) == 0 && tile_class(p, c, 1, kt, kid) == 0)
+            continue;
+          const int sk = kidx % C::kKStages, sv = vidx % C::kVStages;
+          bool got = true;
+          if (lane == 0 && kidx >= C::kKStages)
+            got = mbar_wait_s(BAR(C::bKEmpty + sk), ((kidx / C::kKStages) - 1) & 1, abort_addr);
+          if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(BAR(C::bKFull + sk), C::kTileBytes);
+            for (int x = 0; x < C::kBoxes; ++x)
+              tma_load_3d_s(sKa + sk * C::kTileBytes + x * kBoxBytes, &tm_k, BAR(C::bKFull + sk),
+                          col0 + 64 * x, kt * kBN, z);
           }
+          ++kidx;
+          if (lane == 0 && vidx >= C::kVStages)
+            got = mbar_wait_s(BAR(C::bVEmpty + sv), ((vidx / C::kVStages) - 1) & 1, abort_addr);
+          if (!__shfl_sync(~0u, got, 0)) { ok = false; break; }
+          if (lane == 0) {
+            mbar_arrive_expect_tx(BAR(C::bVFull + sv), C::kTileBytes);
+            for (int x = 0; x < C::kBoxes; ++x)
+              tma_load_3d_s(sVa + sv * C::kTileBytes + x * kBoxBytes, &tm_v, BAR(C::bVFull + sv),
+                          col0 + 64 * x, kt * kBN, z);
+          }
+          ++vidx;
         }
       }
-      if (ok) send_step(kStepEnd);
       if (lane == 0 && ld_shared_volatile(abort_addr)) {
         // Let the copies already in flight land before the CTA exits.
-        for (int u = (ring > C::kStages ? ring - C::kStages : 0); u < ring; ++u)
-          mbar_wait_s(BAR(C::bKvFull + u % C::kStages), (u / C::kStages) & 1, never_abort);
+        for (int u = (kidx > C::kKStages ? kidx - C::kKStages : 0); u < kidx; ++u)
+          mbar_wait_s(BAR(C::bKFull + u % C::kKStages), (u / C::kKStages) & 1, never_abort);
+        for (int u = (vidx > C::kVStages ? vidx - C::kVStages : 0); u < vidx; ++u)
+          mbar_wait_s(BAR(C::bVFull + u % C::kVStages), (u / C::kVStages) & 1, never_abort);
         if (!(p.debug_flags & kDebugWithholdQ))
           for (int t = 0; t < kTiles; ++t)
             if (q_uses[t] > 0) mbar_wait_s(BAR(C::bQFull + t), (q_uses[t] - 1) & 1, never_abort);
       }
       __syncwarp();
-    } else if (warp == kWarpMma) {
+    } else if (warp == 9) {
       // ---------------------------------------------------------- MMA
-      // One thread runs the whole MMA loop: its warp shares a sub-partition
-      // with two busy softmax warps, so the loop is kept to the few
-      // instructions each MMA needs.
-      if (lane == 0) {
-        constexpr uint32_t idesc_qk = idesc_f32acc(128, kBN, 0, 0, kF16);
-        constexpr uint32_t idesc_pv = idesc_f32acc(128, D, 0, 1, kF16);
-        // Operand descriptors as low halves (start address + leading
-        // offset); every operand here has an 8-row stride of 1024 B (common
-        // high half).  Q and K are K-major (64-column boxes); V is N-major
-        // with a box of 64 columns per leading step.  A ring stage s starts
-        // s * kTileBytes after the ring base.
-        constexpr uint32_t kDescHi = sdesc_hi(1024);
-        constexpr uint32_t kStageLo = C::kTileBytes >> 4;
-        const uint32_t q_lo = sdesc_lo(sQa, 16);
-        const uint32_t k_lo = sdesc_lo(sRa, 16);
-        const uint32_t v_lo = sdesc_lo(sRa, kBoxBytes);
-        bool ok = true;
-        int s_cnt0 = 0, s_cnt1 = 0;       // S/P handshakes so far (all items)
-        int o_cnt0 = 0, o_cnt1 = 0;       // O_final commits so far
-        int q_cnt0 = 0, q_cnt1 = 0;       // Q tiles consumed so far
-        // Pending P V per tile: ring stage of V (-1: none), fill parity of
-        // that stage, and flags (bit 0: accumulates into O, bit 1: ends its
-        // item).
-        int pend_v0 = -1, pend_v1 = -1;
-        uint32_t pend_ph0 = 0, pend_ph1 = 0, pend_f0 = 0, pend_f1 = 0;
-        uint32_t v_users = 0;             // pending P V per ring stage (2 bits each)
-        int ring = 0;                     // ring stages consumed so far
+      constexpr uint32_t idesc_qk = idesc_f32acc(128, kBN, 0, 0, kF16);
+      constexpr uint32_t idesc_pv = idesc_f32acc(128, D, 0, 1, kF16);
+      // Operand descriptors as low halves (start address + leading offset);
+      // every operand here has an 8-row stride of 1024 B (common high half).
+      // Q and K are K-major (64-column boxes); V is N-major with a box of
+      // 64 columns per leading step.
+      constexpr uint32_t kDescHi = sdesc_hi(1024);
+      const uint32_t q_lo = sdesc_lo(sQa, 16), k_lo = sdesc_lo(sKa, 16);
+      const uint32_t v_lo = sdesc_lo(sVa, kBoxBytes);
+      bool ok = true;
+      int steps[kTiles] = {0, 0};       // S/P handshakes so far (all items)
+      int pend_idx[kTiles] = {-1, -1};  // K/V index whose P V is still to issue
+      int item_pv[kTiles] = {0, 0};     // P V issued in the current item
+      int o_uses[kTiles] = {0, 0};      // items that produced an O
+      int q_uses[kTiles] = {0, 0};
+      // Outstanding P V per V stage, 4 bits per stage (kept in a register).
+      uint32_t v_users = 0;
 
-        // O_t += P_t V for the pending key tile of tile t.
-        auto issue_pv = [&](int t) -> bool {
-          const int sv = t ? pend_v1 : pend_v0;
-          const uint32_t fl = t ? pend_f1 : pend_f0;
-          const int o_cnt = t ? o_cnt1 : o_cnt0;
-          const int s_cnt = t ? s_cnt1 : s_cnt0;
-          if (!(fl & 1u) && o_cnt > 0 &&
-              !mbar_wait_s(BAR(C::bOEmpty + t), (o_cnt - 1) & 1, abort_addr))
-            return false;  // the previous item's O_t has not been read out yet
-          if (!mbar_wait_s(BAR(C::bPFull + t), (s_cnt - 1) & 1, abort_addr)) return false;
-          if (!mbar_wait_s(BAR(C::bKvFull + sv), t ? pend_ph1 : pend_ph0, abort_addr))
-            return false;
-          tc_fence_after();
-          const uint32_t vd = v_lo + uint32_t(sv) * kStageLo;
-          const uint32_t dO = tmem + C::kColO + t * D, aP = tmem + t * 128;
-          // Rolled: the MMA warp shares its sub-partition (and instruction
-          // cache) with two softmax warps; issue is bound by the tensor pipe
-          // anyway (one MMA per 64 cycles).
-#pragma unroll 1
-          for (int kk = 0; kk < kBN / 16; ++kk)
-            umma_ts_lh(dO, aP + kk * 8, vd + kk * (2048 >> 4), kDescHi, idesc_pv,
-                       (kk > 0 || (fl & 1u)) ? 1u : 0u);
-          v_users -= 1u << (2 * sv);
-          if (((v_users >> (2 * sv)) & 3u) == 0) umma_commit_s(BAR(C::bKvEmpty + sv));
-          if (fl & 2u) {
-            umma_commit_s(BAR(C::bOFinal + t));
-            if (t) ++o_cnt1; else ++o_cnt0;
-          }
-          if (t) pend_v1 = -1; else pend_v0 = -1;
-          return true;
-        };
+      // O_t += P_t V for the key tile whose S_t the softmax has just turned
+      // into P_t.  Issued as soon as P_t is ready so that V stages free up.
+      // Lane 0 only.
+      auto issue_pv = [&](int t) -> bool {
+        const int vi = pend_idx[t];
+        const int sv = vi % C::kVStages;
+        if (item_pv[t] == 0 && o_uses[t] > 0 &&
+            !mbar_wait_s(BAR(C::bOEmpty + t), (o_uses[t] - 1) & 1, abort_addr))
+          return false;  // the previous item's O_t has been read out
+        if (!mbar_wait_s(BAR(C::bPFull + t), (steps[t] - 1) & 1, abort_addr)) return false;
+        if (!mbar_wait_s(BAR(C::bVFull + sv), (vi / C::kVStages) & 1, abort_addr)) return false;
+        tc_fence_after();
+        const uint32_t vd = v_lo + uint32_t(sv) * (C::kTileBytes >> 4);
+        const uint32_t acc0 = item_pv[t] > 0 ? 1u : 0u;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_ts_lh(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8, vd + kk * (2048 >> 4),
+                     kDescHi, idesc_pv, kk > 0 ? 1u : acc0);
+        v_users -= 1u << (4 * sv);
+        if (((v_users >> (4 * sv)) & 15u) == 0) umma_commit_s(BAR(C::bVEmpty + sv));
+        pend_idx[t] = -1;
+        ++item_pv[t];
+        return true;
+      };
 
-        for (int k = 0; ok; ++k) {
-          const int e = k % kStepRing;
-          if (!mbar_wait_s(BAR(C::bStepFull + e), (k / kStepRing) & 1, abort_addr)) {
+      int idx = 0;
+      for (int n = 0; ok; ++n) {
+        const int slot = n % kSchedRing;
+        int w = -1;
+        if (lane == 0) {
+          if (mbar_wait_s(BAR(C::bSchedFull + slot), (n / kSchedRing) & 1, abort_addr)) {
+            w = int(ld_shared_volatile(sched_ids + 4u * slot));
+            mbar_arrive(BAR(C::bSchedEmpty + slot));
+          } else {
             ok = false;
-            break;
           }
-          const uint32_t cmd = ld_shared_volatile(sb + C::kSmemSteps + 4u * e);
-          mbar_arrive(BAR(C::bStepEmpty + e));
-          // The end command visits no tile: the loop below then only issues
-          // the pending P V of the last item.
-          const int sk = ring % C::kStages, sv = (ring + 1) % C::kStages;
-          const uint32_t k_par = (ring / C::kStages) & 1, v_par = ((ring + 1) / C::kStages) & 1;
-          ring += 2;
-          bool have_k = false;
-#pragma unroll 1
-          for (int t = 0; t < kTiles; ++t) {
-            // P V of this tile's previous key tile first: it reads P_t from
-            // the columns that this Q K^T overwrites.  A pending P V is
-            // issued at the next step even when the tile does not visit it,
-            // so that its V stage never waits on a later visit of the tile.
-            if ((t ? pend_v1 : pend_v0) >= 0 && !issue_pv(t)) { ok = false; break; }
-            if (!((cmd >> t) & 1u)) continue;
-            const bool first = (cmd >> (2 + t)) & 1u, is_last = (cmd >> (4 + t)) & 1u;
-            if (first) {
-              if (!mbar_wait_s(BAR(C::bQFull + t), (t ? q_cnt1 : q_cnt0) & 1, abort_addr)) {
-                ok = false;
-                break;
-              }
-              if (t) ++q_cnt1; else ++q_cnt0;
-            }
-            if (!have_k) {
-              if (!mbar_wait_s(BAR(C::bKvFull + sk), k_par, abort_addr)) { ok = false; break; }
-              have_k = true;
-            }
-            tc_fence_after();
-            const uint32_t qd = q_lo + t * (C::kTileBytes >> 4);
-            const uint32_t kd = k_lo + uint32_t(sk) * kStageLo;
-#pragma unroll 1
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
-              umma_ss_lh(tmem + t * 128, qd + off, kDescHi, kd + off, kDescHi, idesc_qk,
-                         kk > 0 ? 1u : 0u);
-            }
-            umma_commit_s(BAR(C::bSFull + t));
-            // Q_t may be reloaded once this item's last Q K^T is done.
-            if (is_last) umma_commit_s(BAR(C::bQEmpty + t));
-            const uint32_t fl = (first ? 0u : 1u) | (is_last ? 2u : 0u);
-            if (t) {
-              ++s_cnt1; pend_v1 = sv; pend_ph1 = v_par; pend_f1 = fl;
-            } else {
-              ++s_cnt0; pend_v0 = sv; pend_ph0 = v_par; pend_f0 = fl;
-            }
-            v_users += 1u << (2 * sv);
-          }
-          if (cmd & kStepEnd) break;
-          // K_kt is free once both Q K^T have read it.
-          if (ok) umma_commit_s(BAR(C::bKvEmpty + sk));
         }
+        ok = __shfl_sync(~0u, ok, 0);
+        w = __shfl_sync(~0u, w, 0);
+        if (!ok || w < 0) break;
+        Item c = make_item(p, w, q_blocks, group, causal);
+        item_query_ids(p, c);
+        // This item's Q tiles (waited even by a tile with no visible key,
+        // so that the phases stay in step with the producer).
+#pragma unroll
+        for (int t = 0; t < kTiles; ++t) {
+          item_pv[t] = 0;
+          if (!has_rows(c, t)) continue;
+          bool got = true;
+          if (lane == 0) got = mbar_wait_s(BAR(C::bQFull + t), q_uses[t] & 1, abort_addr);
+          if (!__shfl_sync(~0u, got, 0)) ok = false;
+          ++q_uses[t];
+        }
+        if (!ok) break;
+        if (lane == 0) tc_fence_after();
+        for (int kt = 0; ok && kt < c.kt_end; ++kt) {
+          const uint32_t kid = key_tile_ids(p, c, kt);
+          const int cls0 = tile_class(p, c, 0, kt, kid);
+          const int cls1 = tile_class(p, c, 1, kt, kid);
+          if (cls0 == 0 && cls1 == 0) continue;
+          if (lane == 0) {
+            const int sk = idx % C::kKStages;
+            if (!mbar_wait_s(BAR(C::bKFull + sk), (idx / C::kKStages) & 1, abort_addr)) {
+              ok = false;
+            } else {
+              tc_fence_after();
+              const uint32_t kd = k_lo + uint32_t(sk) * (C::kTileBytes >> 4);
+#pragma unroll
+              for (int t = 0; t < kTiles; ++t) {
+                if (pend_idx[t] >= 0 && !issue_pv(t)) { ok = false; break; }
+                if ((t == 0 ? cls0 : cls1) == 0) continue;
+                const uint32_t qd = q_lo + t * (C::kTileBytes >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
+                  umma_ss_lh(tmem + t * 128, qd + off, kDescHi, kd + off, kDescHi, idesc_qk,
+                             kk > 0 ? 1u : 0u);
+                }
+                umma_commit_s(BAR(C::bSFull + t));
+                pend_idx[t] = idx;
+                ++steps[t];
+                v_users += 1u << (4 * (idx % C::kVStages));
+              }
+              if (ok) umma_commit_s(BAR(C::bKEmpty + sk));
+            }
+          }
+          ok = __shfl_sync(~0u, ok, 0);
+          ++idx;
+        }
+        if (lane == 0 && ok) {
+#pragma unroll
+          for (int t = 0; t < kTiles; ++t) {
+            if (pend_idx[t] >= 0 && !issue_pv(t)) { ok = false; break; }
+            if (item_pv[t] > 0) {
+              umma_commit_s(BAR(C::bOFinal + t));
+              ++o_uses[t];
+            }
+            // Q_t may be reloaded once this item's Q K^T are done.
+            if (has_rows(c, t)) umma_commit_s(BAR(C::bQEmpty + t));
+          }
+        }
+        ok = __shfl_sync(~0u, ok, 0);
+      }
+      if (lane == 0) {
         // Make sure no MMA is in flight when TMEM is released.
         umma_commit_s(BAR(C::bDrain));
         mbar_wait_s(BAR(C::bDrain), 0, never_abort);
       }
       __syncwarp();
-    }
-  } else if (warp >= kWarpEpi) {
-    reg_dealloc<kRegsEpi>();
-    // ------------------------------------------------------------ epilogue
-    // Warp 8 + q owns TMEM lane quarter q: rows 32 q .. 32 q + 31 of both
-    // query tiles.  The tiles are served independently, each as soon as its
-    // record (from the softmax warps) and, if it has one, its final O (from
-    // the MMA warp) are both ready; lane 0 polls and the warp follows.
-    const int wq = warp - kWarpEpi;
-    const int row = wq * 32 + lane;
-    const uint32_t lane_base = uint32_t(wq * 32) << 16;
-    // Per-tile counters kept as scalars (a run-time tile index into an
-    // array would place it in local memory).
-    int o_cnt0 = 0, o_cnt1 = 0, rec_cnt0 = 0, rec_cnt1 = 0;
-    bool done0 = false, done1 = false;
-    uint64_t idle_since = 0;
-    uint32_t spins = 0;
-    while (!(done0 && done1)) {
-      int pick = -1;
-      if (lane == 0) {
-#pragma unroll
-        for (int t = 0; t < kTiles; ++t) {
-          if (pick >= 0 || (t ? done1 : done0)) continue;
-          if (!mbar_test_wait(BAR(C::bStatsFull + t), (t ? rec_cnt1 : rec_cnt0) & 1)) continue;
-          const uint32_t flags = ld_shared_volatile(rec + t * C::kRecBytes + 12);
-          if ((flags & kRecHaveO) &&
-              !mbar_test_wait(BAR(C::bOFinal + t), (t ? o_cnt1 : o_cnt0) & 1))
-            continue;
-          pick = t;
-        }
-        // Back off between polls so that the idle epilogue warps leave the
-        // issue slots to the softmax warps of the same sub-partitions.
-        if (pick < 0) __nanosleep(256);
-        if (pick < 0 && (++spins & 15u) == 0) {
-          // Bounded like every other wait: give up after one second without
-          // progress, or when another role has raised the abort flag.
-          const uint64_t now = globaltimer_ns();
-          if (idle_since == 0) idle_since = now;
-          if (ld_shared_volatile(abort_addr)) pick = -2;
-          else if (now - idle_since > 1000000000ull) {
-            st_shared_u32(abort_addr, 1u);
-            pick = -2;
-          }
-        }
-        if (pick >= 0) idle_since = 0;
-      }
-      pick = __shfl_sync(~0u, pick, 0);
-      if (pick == -2) break;
-      if (pick < 0) continue;
-      const int t = pick;
-      const int rec_cnt = t ? rec_cnt1 : rec_cnt0;
-      const int o_cnt = t ? o_cnt1 : o_cnt0;
-      // Every lane observes the completed phases itself (acquire).
-      mbar_wait_s(BAR(C::bStatsFull + t), rec_cnt & 1, abort_addr);
-      if (t) ++rec_cnt1; else ++rec_cnt0;
-      const uint32_t rt = rec + t * C::kRecBytes;
-      const int b = int(ld_shared_volatile(rt + 0));
-      const int h = int(ld_shared_volatile(rt + 4));
-      const int q0 = int(ld_shared_volatile(rt + 8));
-      const uint32_t flags = ld_shared_volatile(rt + 12);
-      const float inv = __uint_as_float(ld_shared_volatile(rt + 16 + 4 * row));
-      __syncwarp();
-      mbar_arrive(BAR(C::bStatsEmpty + t));
-      if (flags & kRecDone) {
-        if (t) done1 = true; else done0 = true;
-        continue;
-      }
-      const bool have_o = flags & kRecHaveO;
-      if (have_o) {
-        mbar_wait_s(BAR(C::bOFinal + t), o_cnt & 1, abort_addr);
-        if (t) ++o_cnt1; else ++o_cnt0;
-        tc_fence_after();
-      }
-      const int i = q0 + row;
-      const bool row_real = i < p.Sq;
-      uint16_t* orow = out + b * p.q_sb + h * p.q_sh + int64_t(i) * p.q_ss;
-      const uint32_t tO = tmem + lane_base + C::kColO + t * D;
-      // 16 columns at a time (this warpgroup runs on few registers).
-#pragma unroll 1
-      for (int cc = 0; cc < D / 16; ++cc) {
-        uint32_t orr[16];
-        if (have_o) {
-          tmem_ld16(tO + cc * 16, orr);
-          tmem_ld_wait16(orr);
-          if (cc == D / 16 - 1) {
-            // O_t has been read: the next item's first P V may overwrite it.
-            tc_fence_before();
-            mbar_arrive(BAR(C::bOEmpty + t));
-          }
-        }
-        if (row_real) {
-          uint32_t wv[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float o0 = have_o ? __uint_as_float(orr[2 * e]) * inv : 0.f;
-            const float o1 = have_o ? __uint_as_float(orr[2 * e + 1]) * inv : 0.f;
-            wv[e] = pack_h2<kF16>(o0, o1);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 16);
-          dst[0] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
-          dst[1] = make_uint4(wv[4], wv[5], wv[6], wv[7]);
-        }
-      }
     }
   } else {
     reg_alloc<kRegsSoftmax>();
@@ -798,12 +553,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + C::kColO + t * D;
     const float sl2 = p.scale_log2;
     const bool has_alibi = p.slopes != nullptr;
-    const uint32_t lock = sb + C::kSmemLock + 4 * wq;
-    int steps = 0, st_cnt = 0;
+    int steps = 0, o_uses = 0;
     bool ok = true;
 
     for (int n = 0; ok; ++n) {
-      const int w = read_item<C>(sb, n, abort_addr, ok);
+      const int slot = n % kSchedRing;
+      int w = -1;
+      if (lane == 0) {
+        if (mbar_wait_s(BAR(C::bSchedFull + slot), (n / kSchedRing) & 1, abort_addr)) {
+          w = int(ld_shared_volatile(sched_ids + 4u * slot));
+          mbar_arrive(BAR(C::bSchedEmpty + slot));
+        } else {
+          ok = false;
+        }
+      }
+      ok = __shfl_sync(~0u, ok, 0);
+      w = __shfl_sync(~0u, w, 0);
       if (!ok || w < 0) break;
       Item c = make_item(p, w, q_blocks, group, causal);
       item_query_ids(p, c);
@@ -825,172 +590,86 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t kid = key_tile_ids(p, c, kt);
         const int cls = tile_class(p, c, t, kt, kid);
         if (cls == 0) continue;
+        // Every wait is agreed warp-wide before the .sync.aligned TMEM ops.
+        const bool got_s = mbar_wait_s(BAR(C::bSFull + t), steps & 1, abort_addr);
+        if (!__all_sync(~0u, got_s)) { ok = false; break; }
+        tc_fence_after();
+        const int k0 = kt * kBN;
         // Without a bias and with a positive scale, max(s * c) = c * max(s)
         // exactly, and x - m folds into one fma per element; the same
         // arithmetic is used whether or not the tile needs masking, so the
         // result does not depend on the tile classification.
         const bool plain = !has_alibi && sl2 > 0.f;
         const bool masked = cls == 1;
-        const int k0 = kt * kBN;
-        // Visibility of the 128 keys of this tile for row i, as bits (masked
-        // tiles only).  It does not depend on S, so it is worked out before
-        // the wait.
-        uint32_t vb[4] = {~0u, ~0u, ~0u, ~0u};
+        uint32_t sr[4][32];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, sr[q4]);
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) tmem_ld_wait(sr[q4]);
+        if (!plain) {
+          // x = s * scale * log2(e) + ALiBi, kept in sr
+#pragma unroll
+          for (int e = 0; e < 128; ++e) {
+            float x = __uint_as_float(sr[e >> 5][e & 31]) * sl2;
+            if (has_alibi) x = fmaf(-slope_l2, float(abs(i - (k0 + e))), x);
+            sr[e >> 5][e & 31] = __float_as_uint(x);
+          }
+        }
         if (masked) {
           // Key ids of this tile as id==1 bits (modality rule), by warp votes.
           uint32_t kb[4] = {0u, 0u, 0u, 0u};
-          if (ids) {
+          if (ids && cls == 1) {
 #pragma unroll
             for (int wd = 0; wd < 4; ++wd) {
               const int j = k0 + 32 * wd + lane;
               kb[wd] = __ballot_sync(~0u, j < p.Sk && (ids[j < p.Sk ? j : 0] & 1) == 1);
             }
           }
-          int lim = row_real ? (c.nkeys - 1 - k0) : -1;  // keys e <= lim visible
-          if (causal) lim = min(lim, i - k0);
+          // Visibility of the 128 keys of this tile for row i, as bits.
+          uint32_t vb[4];
+          {
+            int lim = row_real ? (c.nkeys - 1 - k0) : -1;  // keys e <= lim visible
+            if (causal) lim = min(lim, i - k0);
 #pragma unroll
-          for (int wd = 0; wd < 4; ++wd) vb[wd] = range_bits(0, lim, wd);
-          if (mrow) {
-            const uint8_t* mk = mrow + k0;
-            const int nvalid = min(kBN, p.Sk - k0);
-            const bool vec = (reinterpret_cast<uintptr_t>(mk) & 15u) == 0;
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-              uint32_t m = 0;
-              if (vec && 32 * wd + 32 <= nvalid) {
-                // 32 mask bytes as two 16-byte loads, one bit per byte.
-#pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-                  const uint4 a4 = reinterpret_cast<const uint4*>(mk + 32 * wd)[hv];
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    const uint32_t v = q == 0 ? a4.x : (q == 1 ? a4.y : (q == 2 ? a4.z : a4.w));
-                    const int bit = 16 * hv + 4 * q;
-                    m |= ((v & 0xffu) ? 1u : 0u) << bit;
-                    m |= ((v & 0xff00u) ? 1u : 0u) << (bit + 1);
-                    m |= ((v & 0xff0000u) ? 1u : 0u) << (bit + 2);
-                    m |= ((v & 0xff000000u) ? 1u : 0u) << (bit + 3);
-                  }
-                }
-              } else {
-                for (int e = 0; e < 32 && 32 * wd + e < nvalid; ++e)
-                  m |= uint32_t(mk[32 * wd + e] != 0) << e;
+            for (int wd = 0; wd < 4; ++wd) vb[wd] = range_bits(0, lim, wd);
+            if (mrow) {
+#pragma unroll 1
+              for (int wd = 0; wd < 4; ++wd) {
+                uint32_t m = 0;
+                const int jw = k0 + 32 * wd;
+                for (int e = 0; e < 32 && jw + e < p.Sk; ++e)
+                  m |= uint32_t(mrow[jw + e] != 0) << e;
+                vb[wd] &= m;
               }
-              vb[wd] &= m;
             }
-          }
-          if (ids) {
+            if (ids) {
 #pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-              uint32_t m = modality_row_bits(p.allow_bits, id_i, kb[wd], true);
-              if (p.allow_bits & 16u) m |= range_bits(i - k0, i - k0, wd);
-              vb[wd] &= m;
+              for (int wd = 0; wd < 4; ++wd) {
+                uint32_t m = modality_row_bits(p.allow_bits, id_i, kb[wd], true);
+                if (p.allow_bits & 16u) m |= range_bits(i - k0, i - k0, wd);
+                vb[wd] &= m;
+              }
             }
           }
+#pragma unroll
+          for (int e = 0; e < 128; ++e)
+            if (!((vb[e >> 5] >> (e & 31)) & 1u)) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
         }
-        if (!warp_wait(BAR(C::bSFull + t), steps & 1, abort_addr)) { ok = false; break; }
-        tc_fence_after();
-        if (kSoftmaxTurns == 1) turn_acquire(lock, abort_addr);
-        uint32_t sr[4][32];
-        uint32_t ca[32], cb[32];  // S chunks of the exponential phase (reloaded)
-        float mx;
-        if (plain && !masked) {
-          // Row max of the first half while the second half loads.
-          tmem_ld64_wait(tS, sr[0], sr[1]);
-          tmem_ld32(tS + 64, sr[2]);
-          tmem_ld32(tS + 96, sr[3]);
-          if (kSoftmaxTurns == 2) turn_acquire(lock, abort_addr);
-          float mx8[8];
+        // Row max: three-input max, 8 independent chains.
+        float mx8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          mx8[u] = fmaxf(__uint_as_float(sr[0][u]), __uint_as_float(sr[0][u + 8]));
+#pragma unroll
+        for (int e = 16; e < 128; e += 16) {
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            mx8[u] = fmax3(__uint_as_float(sr[0][u]), __uint_as_float(sr[0][u + 8]),
-                           __uint_as_float(sr[0][u + 16]));
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            mx8[u] = fmax3(mx8[u], __uint_as_float(sr[0][u + 24]), __uint_as_float(sr[1][u]));
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            mx8[u] = fmax3(mx8[u], __uint_as_float(sr[1][u + 8]), __uint_as_float(sr[1][u + 16]));
-#pragma unroll
-          for (int u = 0; u < 8; ++u) mx8[u] = fmaxf(mx8[u], __uint_as_float(sr[1][u + 24]));
-          tmem_ld_wait(sr[2]);
-          tmem_ld_wait(sr[3]);
-#pragma unroll
-          for (int h = 2; h < 4; ++h) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              mx8[u] = fmax3(mx8[u], __uint_as_float(sr[h][u]), __uint_as_float(sr[h][u + 8]));
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              mx8[u] = fmax3(mx8[u], __uint_as_float(sr[h][u + 16]),
-                             __uint_as_float(sr[h][u + 24]));
-          }
-          mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                     fmaxf(mx8[6], mx8[7])) * sl2;
-          // The first chunk of the exponential phase is read again from
-          // TMEM (see below); start that load now.
-          tmem_ld32(tS, ca);
-        } else {
-          tmem_ld64_wait(tS, sr[0], sr[1]);
-          tmem_ld64_wait(tS + 64, sr[2], sr[3]);
-          if (kSoftmaxTurns == 2) turn_acquire(lock, abort_addr);
-          if (has_alibi) {
-            // x = s * scale * log2(e) - slope * log2(e) * |i - j|.  Below the
-            // diagonal (j <= i for the whole tile) the bias is
-            // slope_l2 * (k0 - i) + slope_l2 * e, above it the negative of
-            // that: one fma per element for the bias, one for the scale.
-            const int dlo = k0 - i, dhi = k0 + kBN - 1 - i;  // j - i over the tile
-            const uint64_t c2 = f2_pack(sl2, sl2);
-            if (dhi <= 0 || dlo >= 0) {
-              const float g = dhi <= 0 ? slope_l2 : -slope_l2;
-              const float B = g * float(dlo);
-              const uint64_t g2 = f2_pack(g, g), B2 = f2_pack(B, B);
-#pragma unroll
-              for (int e = 0; e < 128; e += 2) {
-                const uint64_t b2 = ffma2(g2, f2_pack(float(e), float(e + 1)), B2);
-                const uint64_t x2 = ffma2(
-                    f2_pack(__uint_as_float(sr[e >> 5][e & 31]),
-                            __uint_as_float(sr[e >> 5][(e & 31) + 1])),
-                    c2, b2);
-                float x0, x1;
-                f2_unpack(x2, x0, x1);
-                sr[e >> 5][e & 31] = __float_as_uint(x0);
-                sr[e >> 5][(e & 31) + 1] = __float_as_uint(x1);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 128; ++e) {
-                const float x = __uint_as_float(sr[e >> 5][e & 31]) * sl2;
-                sr[e >> 5][e & 31] =
-                    __float_as_uint(fmaf(-slope_l2, fabsf(float(dlo + e)), x));
-              }
-            }
-          } else if (!plain) {
-#pragma unroll
-            for (int e = 0; e < 128; ++e)
-              sr[e >> 5][e & 31] = __float_as_uint(__uint_as_float(sr[e >> 5][e & 31]) * sl2);
-          }
-          if (masked) {
-#pragma unroll
-            for (int e = 0; e < 128; ++e)
-              if (!((vb[e >> 5] >> (e & 31)) & 1u)) sr[e >> 5][e & 31] = __float_as_uint(-INFINITY);
-          }
-          // Row max: three-input max, 8 independent chains.
-          float mx8[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u)
-            mx8[u] = fmaxf(__uint_as_float(sr[0][u]), __uint_as_float(sr[0][u + 8]));
-#pragma unroll
-          for (int e = 16; e < 128; e += 16) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              mx8[u] = fmax3(mx8[u], __uint_as_float(sr[(e + u) >> 5][(e + u) & 31]),
-                             __uint_as_float(sr[(e + 8 + u) >> 5][(e + 8 + u) & 31]));
-          }
-          mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
-                     fmaxf(mx8[6], mx8[7]));
-          if (plain) mx *= sl2;  // -inf stays -inf (sl2 > 0)
+            mx8[u] = fmax3(mx8[u], __uint_as_float(sr[(e + u) >> 5][(e + u) & 31]),
+                           __uint_as_float(sr[(e + 8 + u) >> 5][(e + 8 + u) & 31]));
         }
+        float mx = fmax3(fmax3(mx8[0], mx8[1], mx8[2]), fmax3(mx8[3], mx8[4], mx8[5]),
+                         fmaxf(mx8[6], mx8[7]));
+        if (plain) mx *= sl2;  // -inf stays -inf (sl2 > 0)
         // Move the reference max only when it grew by more than 2^8: O and l
         // are then rescaled by alpha (exact after the final division).
         float alpha = 1.f;
@@ -1005,20 +684,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         const uint64_t neg_m = f2_pack(-m_use, -m_use);
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
-        const bool fold = plain;  // scores still unscaled in sr
         uint64_t rs2[4] = {0, 0, 0, 0};  // 4 chains of packed partial sums
-        // P for the 32 keys of chunk q from their scores c (raw scores when
-        // fold, else x in log2 units), written over packed columns
-        // 16q .. 16q+15, and added to the row sum.
-        auto exp_chunk = [&](const uint32_t (&c)[32], int q) {
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const uint64_t s2 = f2_pack(__uint_as_float(c[e]), __uint_as_float(c[e + 1]));
+            const uint64_t s2 = f2_pack(__uint_as_float(sr[q4][e]), __uint_as_float(sr[q4][e + 1]));
             float a0, a1;
-            f2_unpack(fold ? ffma2(s2, sl2x2, neg_m) : fadd2(s2, neg_m), a0, a1);
+            f2_unpack(plain ? ffma2(s2, sl2x2, neg_m) : fadd2(s2, neg_m), a0, a1);
             float p0, p1;
-            if ((kEmuPairs >> (e >> 1)) & 1u) {  // -inf gives 0 on both paths
+            if ((kSoftExpPairs >> (e >> 1)) & 1u) {
               exp2_fma_x2(a0, a1, p0, p1);
             } else {
               p0 = ex2_approx(a0);  // 2^-inf = 0 for masked keys
@@ -1027,27 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             rs2[(e >> 1) & 3] = fadd2(rs2[(e >> 1) & 3], f2_pack(p0, p1));
             pk[e >> 1] = pack_h2<kF16>(p0, p1);
           }
-          tmem_st16(tS + q * 16, pk);
-        };
-        if (plain && !masked) {
-          // The scores are read from TMEM again, 32 keys at a time, in a
-          // rolled loop: the whole step then fits the instruction cache.
-          // Chunk q + 1 loads while chunk q is exponentiated; P of chunk q
-          // lands in columns 16q .. 16q+15, which hold scores of chunks
-          // already read.
-          tmem_ld_wait(ca);
-#pragma unroll 1
-          for (int q = 0; q < 4; q += 2) {
-            tmem_ld32(tS + 32 * (q + 1), cb);
-            exp_chunk(ca, q);
-            tmem_ld_wait(cb);
-            if (q + 2 < 4) tmem_ld32(tS + 32 * (q + 2), ca);
-            exp_chunk(cb, q + 1);
-            if (q + 2 < 4) tmem_ld_wait(ca);
-          }
-        } else {
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) exp_chunk(sr[q4], q4);
+          tmem_st16(tS + q4 * 16, pk);
         }
         if (item_steps > 0 && __any_sync(~0u, rescale)) {
           // S ready implies every earlier MMA (the previous P V) is complete,
@@ -1063,7 +719,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st32(tO + cc * 32, orr);
           }
         }
-        if (kSoftmaxTurns) turn_release(lock);
         float r[8];
 #pragma unroll
         for (int u = 0; u < 4; ++u) f2_unpack(rs2[u], r[2 * u], r[2 * u + 1]);
@@ -1076,53 +731,56 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
 
-      // The item's record for the epilogue warps (1 / l per row), and the
-      // LSE.
+      // -------------------------------------------------------- epilogue
+      bool have_o = false;
+      if (item_steps > 0) {
+        have_o = __all_sync(~0u, mbar_wait_s(BAR(C::bOFinal + t), o_uses & 1, abort_addr));
+        if (!have_o) { ok = false; break; }
+        ++o_uses;
+        tc_fence_after();
+      }
       const bool empty = !(l > 0.f);
-      if (!publish_record<C>(sb, rec, t, row, st_cnt, abort_addr, c.b, c.h, item_q0(c, t),
-                             item_steps > 0 ? kRecHaveO : 0u, empty ? 0.f : 1.f / l)) {
-        ok = false;
-        break;
+      const float inv = empty ? 0.f : 1.f / l;
+      uint16_t* orow = out + c.b * p.q_sb + c.h * p.q_sh + int64_t(i) * p.q_ss;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t orr[32];
+        if (have_o) {
+          tmem_ld32(tO + cc * 32, orr);
+          tmem_ld_wait(orr);
+          if (cc == D / 32 - 1) {
+            // O_t has been read: the next item's first P V may overwrite it.
+            tc_fence_before();
+            mbar_arrive(BAR(C::bOEmpty + t));
+          }
+        }
+        if (row_real) {
+          uint32_t wv[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float o0 = (have_o && !empty) ? __uint_as_float(orr[2 * e]) * inv : 0.f;
+            const float o1 = (have_o && !empty) ? __uint_as_float(orr[2 * e + 1]) * inv : 0.f;
+            wv[e] = pack_h2<kF16>(o0, o1);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(wv[4 * e], wv[4 * e + 1], wv[4 * e + 2], wv[4 * e + 3]);
+        }
       }
       if (row_real)
         lse[(int64_t(c.b) * p.N + c.h) * p.Sq + i] =
             empty ? -INFINITY : (m_ref + __log2f(l)) * kLn2;
     }
-    // No more items for this tile (skipped after an abort: the epilogue
-    // warps stop on the abort flag).
-    if (ok) publish_record<C>(sb, rec, t, row, st_cnt, abort_addr, 0, 0, 0, kRecDone, 0.f);
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == kWarpMma) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
   if (tid == 0 && ld_shared_volatile(abort_addr)) atomicOr(p.status, 1u);
-}
-
-// Per-device, per-instantiation launch set-up done once: the shared-memory
-// opt-in and the check that the compiled kernel has the launch register
-// count the register split assumes (an increase beyond the launch
-// allocation would wait forever).
-template <int D, bool kF16>
-cudaError_t prepare_once() {
-  static std::atomic<uint64_t> done{0};  // bit per device
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const uint64_t bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
-  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
-  using C = FwdCfg<D>;
-  e = cudaFuncSetAttribute(fwd_sm100<D, kF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  cudaFuncAttributes fa_attr;
-  if ((e = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16>)) != cudaSuccess) return e;
-  if (fa_attr.numRegs < int(kRegsLaunch)) return cudaErrorInvalidConfiguration;
-  done.fetch_or(bit, std::memory_order_acq_rel);
-  return cudaSuccess;
 }
 
 }  // namespace
@@ -1137,7 +795,19 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   if ((e = make_operand_map(&tk, k, p, p.Sk, 128)) != cudaSuccess) return e;
   if ((e = make_operand_map(&tv, v, p, p.Sk, 128)) != cudaSuccess) return e;
   using C = FwdCfg<D>;
-  if ((e = prepare_once<D, kF16>()) != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(fwd_sm100<D, kF16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  // The register split (setmaxnreg) draws on the launch allocation; a build
+  // with fewer registers per thread would leave the increase waiting.
+  static int regs_ok[2][2] = {{0, 0}, {0, 0}};
+  if (!regs_ok[kF16][D == 128]) {
+    cudaFuncAttributes fa_attr;
+    if ((e = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16>)) != cudaSuccess) return e;
+    if (fa_attr.numRegs < int(kRegsLaunch)) return cudaErrorInvalidConfiguration;
+    regs_ok[kF16][D == 128] = 1;
+  }
   const int q_blocks = (p.Sq + kRows - 1) / kRows;
   const int64_t items = int64_t(q_blocks) * p.B * p.N;
   if (items > 0x7fffffff) return cudaErrorInvalidValue;
