@@ -376,6 +376,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float slope_l2 = p.slopes ? p.slopes[c.h] * kLog2e : 0.f;
     const bool has_alibi = p.slopes != nullptr;
     const bool causal = p.mask_flags & FA_MASK_CAUSAL;
+    const bool fold = has_alibi && causal;  // ALiBi linear in i - j
+    const float abs_g = fold ? 0.f : -slope_l2;  // |i - j| form otherwise
     const int32_t* ids = (p.mask_flags & FA_MASK_MODALITY) ? p.ids + int64_t(c.b) * p.Sk : nullptr;
     const int id_j = (ids && j < p.Sk) ? (ids[j] & 1) : 0;
     const int64_t row_base = (int64_t(c.b) * p.N + c.h) * p.Sq;
@@ -393,13 +395,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // -Delta, in this warp's own shared buffer (read back as broadcasts).
       // st[0..63] = -LSE * log2(e), st[64..127] = -Delta (plain shared memory
       // accesses, so the compiler can schedule the broadcast loads freely).
+      // Under the causal rule the ALiBi bias of a visible pair is
+      // -slope * (i - j) = -slope * e - slope * (q0 - j): the column part
+      // -slope * log2(e) * e joins -LSE here, the row part is added below.
       const uint32_t st_w = sb + C::kSmemStats + warp * 2 * kBM * 4;
+      const float col_g = fold ? -slope_l2 : 0.f;
       __syncwarp();
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int i = q0 + 32 * u + lane;
         st_shared_f32(st_w + 4 * (32 * u + lane),
-                      i < p.Sq ? -lse[row_base + i] * kLog2e : -INFINITY);
+                      i < p.Sq ? fmaf(col_g, float(32 * u + lane), -lse[row_base + i] * kLog2e)
+                               : -INFINITY);
         st_shared_f32(st_w + 4 * (kBM + 32 * u + lane), i < p.Sq ? -delta[row_base + i] : 0.f);
       }
       __syncwarp();
@@ -435,7 +442,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(~0u, got_s)) { ok = false; return false; }
       tc_fence_after();
       // P^T = 2^(s * scale * log2 e + bias - LSE) for the 64 queries.
-      const bool plain = cls == 2 && !has_alibi;
+      // The per-element loop runs for masked tiles and for the ALiBi bias
+      // without the causal rule (|i - j| changes sign inside a tile).
+      const bool plain = cls == 2 && (!has_alibi || causal);
       const uint64_t sl2x2 = f2_pack(sl2, sl2);
       float pf[64];
       {
@@ -444,24 +453,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(tb + 32, sr[1]);
         tmem_ld_wait(sr[0]);
         tmem_ld_wait(sr[1]);
-        // x = s * scale * log2(e) - LSE, in place (branch-free)
+        // x = s * scale * log2(e) - LSE (+ the causal ALiBi bias, its row
+        // part -slope * log2(e) * (q0 - j) added here), in place
+        const float brow = -slope_l2 * float(q0 - j);
+        const uint64_t brow2 = f2_pack(brow, brow);
 #pragma unroll
         for (int e = 0; e < kBM; e += 2) {
           const float2 nl = ld_shared_f2(st + 4 * e);
+          uint64_t off2 = f2_pack(nl.x, nl.y);
+          if (fold) off2 = fadd2(off2, brow2);
           float x0, x1;
           f2_unpack(ffma2(f2_pack(__uint_as_float(sr[e >> 5][e & 31]),
                                   __uint_as_float(sr[e >> 5][(e & 31) + 1])),
-                          sl2x2, f2_pack(nl.x, nl.y)),
+                          sl2x2, off2),
                     x0, x1);
           sr[e >> 5][e & 31] = __float_as_uint(x0);
           sr[e >> 5][(e & 31) + 1] = __float_as_uint(x1);
         }
         if (!plain) {
-          // ALiBi bias and the mask, in a loop of their own
+          // The ALiBi bias without the causal rule, and the mask, in a loop
+          // of their own
 #pragma unroll
           for (int e = 0; e < kBM; ++e) {
             float x = __uint_as_float(sr[e >> 5][e & 31]);
-            if (has_alibi) x = fmaf(-slope_l2, float(abs(q0 + e - j)), x);
+            if (has_alibi) x = fmaf(abs_g, float(abs(q0 + e - j)), x);
             if (!((vb[e >> 5] >> (e & 31)) & 1u)) x = -INFINITY;
             sr[e >> 5][e & 31] = __float_as_uint(x);
           }

@@ -134,6 +134,7 @@ struct Item {
   int q0[kTiles], q_last[kTiles];  // q_last < q0 when the tile has no row
   int nkeys;                       // keys allowed by padding / Sk
   int kt_end;                      // one past the last key tile worth visiting
+  int kt_pivot;                    // key tiles visited from here down first, or -1
   uint32_t q_ids[kTiles];          // modality: bit a set if some row has id a
 };
 
@@ -149,6 +150,14 @@ __device__ __forceinline__ uint32_t item_q_ids(const Item& c, int t) {
 }
 __device__ __forceinline__ bool has_rows(const Item& c, int t) {
   return item_q_last(c, t) >= item_q0(c, t);
+}
+
+// Key tile of visit number it.  With an ALiBi bias the scores grow toward
+// the diagonal, so the tiles are visited from the diagonal outward (down to
+// tile 0, then the ones above): the running max is set by the first tile
+// and O is rarely rescaled.  Otherwise in ascending order.
+__device__ __forceinline__ int kt_at(const Item& c, int it) {
+  return it <= c.kt_pivot ? c.kt_pivot - it : it;
 }
 
 // Work item number idx of the claim order.  Heads are taken in groups of
@@ -182,6 +191,7 @@ __device__ __forceinline__ Item make_item(const Problem& p, int idx, int q_block
       c.kt_end = max(c.kt_end, e);
     }
   }
+  c.kt_pivot = p.slopes ? min(c.kt_end - 1, (qb * kRows + kRows - 1) / kBN) : -1;
   return c;
 }
 
@@ -373,7 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           ++q_uses[t];
         }
-        for (int kt = 0; ok && kt < c.kt_end; ++kt) {
+        for (int it = 0; ok && it < c.kt_end; ++it) {
+          const int kt = kt_at(c, it);
           const uint32_t kid = key_tile_ids(p, c, kt);
           if (tile_class(p, c, 0, kt, kid) == 0 && tile_class(p, c, 1, kt, kid) == 0)
             continue;
@@ -487,7 +498,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         if (lane == 0) tc_fence_after();
-        for (int kt = 0; ok && kt < c.kt_end; ++kt) {
+        for (int it = 0; ok && it < c.kt_end; ++it) {
+          const int kt = kt_at(c, it);
           const uint32_t kid = key_tile_ids(p, c, kt);
           const int cls0 = tile_class(p, c, 0, kt, kid);
           const int cls1 = tile_class(p, c, 1, kt, kid);
@@ -586,7 +598,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       float l = 0.f;
       int item_steps = 0;
 
-      for (int kt = 0; kt < c.kt_end; ++kt) {
+      for (int it = 0; it < c.kt_end; ++it) {
+        const int kt = kt_at(c, it);
         const uint32_t kid = key_tile_ids(p, c, kt);
         const int cls = tile_class(p, c, t, kt, kid);
         if (cls == 0) continue;
@@ -607,12 +620,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) tmem_ld_wait(sr[q4]);
         if (!plain) {
-          // x = s * scale * log2(e) + ALiBi, kept in sr
+          // x = s * scale * log2(e) + ALiBi, kept in sr.  The bias
+          // -slope * log2(e) * |i - j| is linear in the key column e when
+          // the tile lies on one side of the diagonal, and under the causal
+          // rule on every tile (the keys j > i are masked to -inf below):
+          // slope_l2 * (j - i) = g * e + g * (k0 - i).  One packed fma per
+          // pair gives the bias, one the scaled score.
+          const int dlo = k0 - i, dhi = k0 + kBN - 1 - i;  // j - i over the tile
+          if (has_alibi && (causal || dhi <= 0 || dlo >= 0)) {
+            const float g = (causal || dhi <= 0) ? slope_l2 : -slope_l2;
+            const uint64_t g2 = f2_pack(g, g), B2 = f2_pack(g * float(dlo), g * float(dlo));
+            const uint64_t c2 = f2_pack(sl2, sl2);
 #pragma unroll
-          for (int e = 0; e < 128; ++e) {
-            float x = __uint_as_float(sr[e >> 5][e & 31]) * sl2;
-            if (has_alibi) x = fmaf(-slope_l2, float(abs(i - (k0 + e))), x);
-            sr[e >> 5][e & 31] = __float_as_uint(x);
+            for (int e = 0; e < 128; e += 2) {
+              const uint64_t b2 = ffma2(g2, f2_pack(float(e), float(e + 1)), B2);
+              float x0, x1;
+              f2_unpack(ffma2(f2_pack(__uint_as_float(sr[e >> 5][e & 31]),
+                                      __uint_as_float(sr[e >> 5][(e & 31) + 1])),
+                              c2, b2),
+                        x0, x1);
+              sr[e >> 5][e & 31] = __float_as_uint(x0);
+              sr[e >> 5][(e & 31) + 1] = __float_as_uint(x1);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 128; ++e) {
+              float x = __uint_as_float(sr[e >> 5][e & 31]) * sl2;
+              if (has_alibi) x = fmaf(-slope_l2, fabsf(float(dlo + e)), x);
+              sr[e >> 5][e & 31] = __float_as_uint(x);
+            }
           }
         }
         if (masked) {

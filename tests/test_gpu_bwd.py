@@ -43,6 +43,13 @@ def test_bf16_causal_alibi(D, S):
     check_bwd(c)
 
 
+@pytest.mark.parametrize("D,sq,sk", [(64, 200, 130), (128, 300, 420)])
+def test_bf16_alibi_no_causal(D, sq, sk):
+    # |i - j| changes sign inside the diagonal tiles: per-element bias there
+    c = I.make_case(f"bwd_anc_D{D}_{sq}x{sk}", 1, 3, sq, sk, D, seed=39, alibi=True)
+    check_bwd(c)
+
+
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("S", [128, 300])
 def test_bf16_causal_no_alibi(D, S):

@@ -53,8 +53,10 @@ def test_bf16_causal_alibi(D):
     check_fwd(c)
 
 
-def test_bf16_alibi_no_causal():
-    c = I.make_case("alibi_nc", 1, 4, 200, 260, 64, seed=14, alibi=True)
+@pytest.mark.parametrize("D,sq,sk", [(64, 200, 260), (128, 700, 650), (64, 300, 900)])
+def test_bf16_alibi_no_causal(D, sq, sk):
+    # key tiles on both sides of the diagonal, visited from it outward
+    c = I.make_case(f"alibi_nc_D{D}_{sq}x{sk}", 1, 4, sq, sk, D, seed=14, alibi=True)
     check_fwd(c)
 
 
