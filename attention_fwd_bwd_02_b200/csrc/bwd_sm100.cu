@@ -587,21 +587,24 @@ cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
   if ((e = make_f32_rows_map(&tdq, dq_acc, p.D, p.Sq, int64_t(p.B) * p.N, C::kDqCols,
                              C::kDqRows)) != cudaSuccess)
     return e;
-  e = cudaFuncSetAttribute(bwd_sm100<D, kF16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  // The register split (setmaxnreg) draws on the launch allocation of
+  // Shared-memory opt-in and the register check, once per device.  The
+  // register split (setmaxnreg) draws on the launch allocation of
   // 65536 / kThreads registers per thread; a build with fewer would leave
   // the increase waiting.
-  static int regs_ok[2][2] = {{0, 0}, {0, 0}};
-  if (!regs_ok[kF16][D == 128]) {
+  static std::atomic<uint64_t> ready{0};
+  e = once_per_device(ready, []() -> cudaError_t {
+    cudaError_t r = cudaFuncSetAttribute(bwd_sm100<D, kF16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (r != cudaSuccess) return r;
     cudaFuncAttributes fa_attr;
-    if ((e = cudaFuncGetAttributes(&fa_attr, bwd_sm100<D, kF16>)) != cudaSuccess) return e;
-    if (fa_attr.numRegs * kThreads < 2 * 128 * int(kRegsSoftmax) + 128 * int(kRegsDq) +
-                                         128 * int(kRegsControl))
-      return cudaErrorInvalidConfiguration;
-    regs_ok[kF16][D == 128] = 1;
-  }
+    if ((r = cudaFuncGetAttributes(&fa_attr, bwd_sm100<D, kF16>)) != cudaSuccess) return r;
+    return fa_attr.numRegs * kThreads <
+                   2 * 128 * int(kRegsSoftmax) + 128 * int(kRegsDq) + 128 * int(kRegsControl)
+               ? cudaErrorInvalidConfiguration
+               : cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
   dim3 grid((p.Sk + kBN - 1) / kBN, p.N, p.B);
   bwd_sm100<D, kF16><<<grid, kThreads, C::kSmemBytes, st>>>(
       tq, tk, tv, tdo, tdq, p, lse, delta, static_cast<uint16_t*>(dk),

@@ -831,19 +831,20 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   if ((e = make_operand_map(&tk, k, p, p.Sk, 128)) != cudaSuccess) return e;
   if ((e = make_operand_map(&tv, v, p, p.Sk, 128)) != cudaSuccess) return e;
   using C = FwdCfg<D>;
-  e = cudaFuncSetAttribute(fwd_sm100<D, kF16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  // The register split (setmaxnreg) draws on the launch allocation; a build
+  // Shared-memory opt-in and the register check, once per device.  The
+  // register split (setmaxnreg) draws on the launch allocation; a build
   // with fewer registers per thread would leave the increase waiting.
-  static int regs_ok[2][2] = {{0, 0}, {0, 0}};
-  if (!regs_ok[kF16][D == 128]) {
+  static std::atomic<uint64_t> ready{0};
+  e = once_per_device(ready, []() -> cudaError_t {
+    cudaError_t r = cudaFuncSetAttribute(fwd_sm100<D, kF16>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (r != cudaSuccess) return r;
     cudaFuncAttributes fa_attr;
-    if ((e = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16>)) != cudaSuccess) return e;
-    if (fa_attr.numRegs < int(kRegsLaunch)) return cudaErrorInvalidConfiguration;
-    regs_ok[kF16][D == 128] = 1;
-  }
+    if ((r = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16>)) != cudaSuccess) return r;
+    return fa_attr.numRegs < int(kRegsLaunch) ? cudaErrorInvalidConfiguration : cudaSuccess;
+  });
+  if (e != cudaSuccess) return e;
   const int q_blocks = (p.Sq + kRows - 1) / kRows;
   const int64_t items = int64_t(q_blocks) * p.B * p.N;
   if (items > 0x7fffffff) return cudaErrorInvalidValue;

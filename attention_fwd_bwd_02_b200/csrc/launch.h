@@ -3,6 +3,9 @@
 
 #include <cuda_runtime.h>
 
+#include <atomic>
+#include <cstdint>
+
 #include "fa_common.cuh"
 
 namespace fa {
@@ -33,6 +36,22 @@ cudaError_t launch_bwd_sm100(const Problem& p, const void* q, const void* k,
 unsigned int* work_counter();
 cudaError_t reset_work_counters();
 int sm_count();
+
+// Runs setup() (function attributes, launch checks) until it succeeds once
+// on the current device; `done` holds one bit per device (devices 0..63;
+// beyond that setup() runs every time).  Two threads may both run setup()
+// the first time, so it must be idempotent.
+template <typename F>
+cudaError_t once_per_device(std::atomic<uint64_t>& done, F&& setup) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = setup();
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
 
 // Helpers (aux.cu), for tensors of element type `elem`.
 enum class Elem { kF32, kBF16, kF16 };

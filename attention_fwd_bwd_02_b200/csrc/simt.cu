@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <atomic>
+
 #include "fa_common.cuh"
 #include "launch.h"
 
@@ -256,8 +258,11 @@ cudaError_t launch_bwd_f32(const Problem& p, const void* q, const void* k,
   const size_t smem = sizeof(float) * (2 * kSimtKeys * (kMaxD + 1) +
                                        2 * kSimtKeys * kMaxD +
                                        kBwdWarps * 2 * kMaxD);
-  cudaError_t e = cudaFuncSetAttribute(
-      bwd_f32_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  static std::atomic<uint64_t> ready{0};
+  cudaError_t e = once_per_device(ready, [smem]() {
+    return cudaFuncSetAttribute(bwd_f32_simt, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(smem));
+  });
   if (e != cudaSuccess) return e;
   dim3 grid((p.Sk + kSimtKeys - 1) / kSimtKeys, p.N, p.B);
   bwd_f32_simt<<<grid, kBwdWarps * 32, smem, st>>>(

@@ -29,12 +29,69 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
+// Encoded maps of recent calls.  A map is a pure function of the encode
+// arguments (address, extents, strides, box, type, swizzle), so an entry
+// stays valid whatever happens to the memory it names; a repeated call with
+// the same tensors skips the encode.
+struct MapArgs {
+  const void* base;
+  cuuint64_t dims[3], strides[2];
+  cuuint32_t box[3];
+  int dtype, swizzle;
+  bool operator==(const MapArgs& o) const {
+    return base == o.base && dims[0] == o.dims[0] && dims[1] == o.dims[1] &&
+           dims[2] == o.dims[2] && strides[0] == o.strides[0] &&
+           strides[1] == o.strides[1] && box[0] == o.box[0] && box[1] == o.box[1] &&
+           box[2] == o.box[2] && dtype == o.dtype && swizzle == o.swizzle;
+  }
+};
+
+constexpr int kMapCacheSlots = 64;
+std::mutex g_map_mu;
+MapArgs g_map_args[kMapCacheSlots];
+CUtensorMap g_maps[kMapCacheSlots];
+int g_map_used = 0, g_map_next = 0;
+
+// Rank-3 tiled map with unit element strides, no interleave, 256-byte L2
+// promotion and zero fill, from the cache or freshly encoded.
+cudaError_t encode_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                      const cuuint64_t dims[3], const cuuint64_t strides[2],
+                      const cuuint32_t box[3], CUtensorMapSwizzle swizzle) {
+  MapArgs a;
+  a.base = base;
+  for (int i = 0; i < 3; ++i) a.dims[i] = dims[i], a.box[i] = box[i];
+  a.strides[0] = strides[0];
+  a.strides[1] = strides[1];
+  a.dtype = int(dtype);
+  a.swizzle = int(swizzle);
+  {
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    for (int i = 0; i < g_map_used; ++i)
+      if (g_map_args[i] == a) {
+        *map = g_maps[i];
+        return cudaSuccess;
+      }
+  }
+  EncodeTiledFn enc = get_encode();
+  if (!enc) return cudaErrorNotSupported;
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  std::lock_guard<std::mutex> lock(g_map_mu);
+  const int slot = g_map_next;  // round robin over the slots
+  g_map_next = (g_map_next + 1) % kMapCacheSlots;
+  if (g_map_used < kMapCacheSlots) ++g_map_used;
+  g_map_args[slot] = a;
+  g_maps[slot] = *map;
+  return cudaSuccess;
+}
+
 }  // namespace
 
 cudaError_t make_operand_map(CUtensorMap* map, const void* base,
                              const Problem& p, int S, int box_rows) {
-  EncodeTiledFn enc = get_encode();
-  if (!enc) return cudaErrorNotSupported;
   cuuint64_t dims[3], strides[2];
   const cuuint64_t esz = 2;  // bf16 or fp16
   if (p.layout == FA_LAYOUT_BSH) {
@@ -51,29 +108,18 @@ cudaError_t make_operand_map(CUtensorMap* map, const void* base,
     strides[1] = dims[0] * dims[1] * esz;
   }
   const cuuint32_t box[3] = {64u, cuuint32_t(box_rows), 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = enc(map, p.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
-                   const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  return encode_3d(map, p.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 cudaError_t make_f32_rows_map(CUtensorMap* map, const void* base, int cols,
                               int rows, int64_t planes, int box_cols,
                               int box_rows) {
-  EncodeTiledFn enc = get_encode();
-  if (!enc) return cudaErrorNotSupported;
   const cuuint64_t dims[3] = {cuuint64_t(cols), cuuint64_t(rows), cuuint64_t(planes)};
   const cuuint64_t strides[2] = {cuuint64_t(cols) * 4, cuuint64_t(cols) * rows * 4};
   const cuuint32_t box[3] = {cuuint32_t(box_cols), cuuint32_t(box_rows), 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base),
-                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  return encode_3d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 }  // namespace fa

@@ -12,6 +12,7 @@ input_layout, pse, padding mask, atten_mask, scale, keep_prob.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import re
@@ -131,6 +132,17 @@ def _ptr(t: Optional[torch.Tensor]):
 
 def _stream(t: torch.Tensor):
     return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+_NULL_CTX = contextlib.nullcontext()
+
+
+def _on_device(dev):
+    """Makes `dev` current for the call (no-op when it already is)."""
+    dev = torch.device(dev)
+    if dev.index is None or dev.index == torch.cuda.current_device():
+        return _NULL_CTX
+    return torch.cuda.device(dev)
 
 
 def _dtype_code(dt):
@@ -267,7 +279,7 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
         lse = torch.empty((shape.B, shape.N, shape.Sq), dtype=torch.float32,
                           device=query.device)
     entry = lib().fa_testing_fwd_withhold_q if _withhold_q else lib().fa_fwd
-    with torch.cuda.device(query.device):
+    with _on_device(query.device):
         st = entry(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
                    None if ps is None else ctypes.byref(ps),
                    None if m is None else ctypes.byref(m),
@@ -312,7 +324,7 @@ def bwd(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
     dq = torch.empty_like(query) if dq is None else dq
     dk = torch.empty_like(key) if dk is None else dk
     dv = torch.empty_like(value) if dv is None else dv
-    with torch.cuda.device(query.device):
+    with _on_device(query.device):
         st = lib().fa_bwd(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
                           _ptr(out), _ptr(dout), _ptr(lse),
                           None if ps is None else ctypes.byref(ps),
@@ -349,7 +361,7 @@ def bwd_noalloc(query, key, value, out, dout, lse, head_num=None, input_layout="
     dq = torch.empty_like(query) if dq is None else dq
     dk = torch.empty_like(key) if dk is None else dk
     dv = torch.empty_like(value) if dv is None else dv
-    with torch.cuda.device(query.device):
+    with _on_device(query.device):
         st = lib().fa_bwd_noalloc(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
                                   _ptr(out), _ptr(dout), _ptr(lse),
                                   None if ps is None else ctypes.byref(ps),
@@ -367,7 +379,7 @@ def build_tile_map(atten_mask, query, key, head_num=None, input_layout="BNSD"):
     m = make_mask(shape, atten_mask=atten_mask, keep=keep)
     n = int(lib().fa_mask_tile_map_size(ctypes.byref(shape), ctypes.byref(m)))
     tm = torch.empty(max(n, 1), dtype=torch.uint8, device=query.device)
-    with torch.cuda.device(query.device):
+    with _on_device(query.device):
         st = lib().fa_build_mask_tile_map(ctypes.byref(shape), ctypes.byref(m),
                                           _ptr(tm), _stream(query))
     _check(st, "fa_build_mask_tile_map")
@@ -383,7 +395,7 @@ def build_modality_mask(modality_ids, allow=((1, 1), (0, 1)), allow_diag=False):
     for a in range(2):
         for c in range(2):
             tab[a][c] = 1 if allow[a][c] else 0
-    with torch.cuda.device(ids.device):
+    with _on_device(ids.device):
         st = lib().fa_build_modality_mask(int(B), int(S), _ptr(ids), ctypes.byref(tab),
                                           1 if allow_diag else 0, _ptr(mask), _stream(ids))
     _check(st, "fa_build_modality_mask")
@@ -393,6 +405,6 @@ def build_modality_mask(modality_ids, allow=((1, 1), (0, 1)), allow_diag=False):
 def sync_status(device=None):
     """Synchronise the current stream and raise if a kernel timed out."""
     dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
-    with torch.cuda.device(dev):
+    with _on_device(dev):
         st = lib().fa_sync_status(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream))
     _check(st, "fa_sync_status")

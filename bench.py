@@ -541,12 +541,18 @@ def run_configs(args):
         bwd = lambda: fa.bwd(q, k, v, out, do, lse, c.N, c.layout, workspace=ws, **kw)
 
         def timed(fn, reps=30, warm=10):
+            """(device ms, call ms): the device time of one call, with the
+            call queued behind a GPU spin so that the host's marshalling
+            and launch cost stay off the events; and the time per call of
+            back-to-back calls, which includes that host cost when it
+            exceeds the device time."""
             for _ in range(warm):
                 fn()
             ts = []
             for _ in range(reps):
                 if do_flush:
                     flush.fill_(1)
+                torch.cuda._sleep(1_000_000)  # about 0.5 ms of GPU spin
                 e0 = torch.cuda.Event(enable_timing=True)
                 e1 = torch.cuda.Event(enable_timing=True)
                 e0.record()
@@ -554,10 +560,15 @@ def run_configs(args):
                 e1.record()
                 torch.cuda.synchronize()
                 ts.append(e0.elapsed_time(e1))
-            return st.median(ts)
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            for _ in range(reps):
+                fn()
+            torch.cuda.synchronize()
+            return st.median(ts), (time.perf_counter() - t0) * 1e3 / reps
 
-        f_ms = timed(fwd)
-        b_ms = timed(bwd)
+        f_ms, f_call = timed(fwd)
+        b_ms, b_call = timed(bwd)
         fa.sync_status()
         nominal = 4.0 * c.B * c.N * c.Sq * c.Sk * c.D / (2.0 if c.causal else 1.0)
         allowed = 4.0 * c.D * _allowed_pairs(c)
@@ -568,6 +579,7 @@ def run_configs(args):
         line = {"metric": METRIC, "config": c.name, "label": label,
                 "dtype": {torch.bfloat16: "bf16", torch.float32: "f32"}[q.dtype],
                 "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4),
+                "fwd_call_ms": round(f_call, 4), "bwd_call_ms": round(b_call, 4),
                 "fwd_tflops": round(nominal / (f_ms * 1e-3) / 1e12, 2),
                 "fwd_tflops_allowed_pairs": round(allowed / (f_ms * 1e-3) / 1e12, 2),
                 "bwd_tflops": round(2.5 * nominal / (b_ms * 1e-3) / 1e12, 2),
@@ -576,7 +588,10 @@ def run_configs(args):
                 "fwd_gbs": round(fwd_bytes / (f_ms * 1e-3) / 1e9, 1),
                 "bwd_gbs": round(bwd_bytes / (b_ms * 1e-3) / 1e9, 1),
                 "peak": peak, "peak_kind": f"{pk_kind} bf16_tflops (burst)",
-                "l2_flushed_between_reps": do_flush, "timing": "median of 30 after 10 warm-ups"}
+                "l2_flushed_between_reps": do_flush,
+                "timing": "fwd_ms/bwd_ms: device time, median of 30 after 10 warm-ups, each call "
+                          "queued behind a GPU spin; *_call_ms: back-to-back calls incl. host cost "
+                          "(no L2 flush)"}
         print(json.dumps(line), flush=True)
         del dev, out, lse, ws
 
