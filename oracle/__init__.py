@@ -53,6 +53,10 @@ class _Mask(ctypes.Structure):
         ("allow10", ctypes.c_int),
         ("allow11", ctypes.c_int),
         ("allow_diag", ctypes.c_int),
+        ("add", ctypes.c_void_p),
+        ("asb", ctypes.c_int64),
+        ("ash", ctypes.c_int64),
+        ("asq", ctypes.c_int64),
     ]
 
 
@@ -156,7 +160,7 @@ class _MaskHolder:
     """Keeps the numpy buffers a _Mask points to alive."""
 
     def __init__(self, B, N, Sq, Sk, causal, kv_len, mask, modality_ids,
-                 allow, allow_diag):
+                 allow, allow_diag, bias=None):
         self.m = _Mask()
         self.m.causal = 1 if causal else 0
         self.keep = []
@@ -190,6 +194,13 @@ class _MaskHolder:
             self.m.allow00, self.m.allow01 = int(a[0, 0]), int(a[0, 1])
             self.m.allow10, self.m.allow11 = int(a[1, 0]), int(a[1, 1])
             self.m.allow_diag = 1 if allow_diag else 0
+        if bias is not None:
+            a = _f64(bias)
+            a4 = np.ascontiguousarray(np.broadcast_to(
+                a.reshape((1,) * (4 - a.ndim) + a.shape), (B, N, Sq, Sk)))
+            self.keep.append(a4)
+            self.m.add = a4.ctypes.data
+            self.m.asb, self.m.ash, self.m.asq = N * Sq * Sk, Sq * Sk, Sk
 
 
 def _prep(q, k, v, n_heads, layout):
@@ -205,17 +216,19 @@ def _prep(q, k, v, n_heads, layout):
 
 def fwd(q, k, v, scale, *, n_heads=None, layout="BNSD", causal=False,
         kv_len=None, mask=None, modality_ids=None, allow=((1, 1), (0, 1)),
-        allow_diag=False, slopes=None):
+        allow_diag=False, slopes=None, bias=None):
     """Attention forward in fp64.  Returns (out, lse) as numpy arrays.
 
     ``out`` has the layout of ``q``; ``lse`` is [B, N, Sq] (natural log,
     -inf for rows with no allowed key).  ``mask`` is a bool/uint8 array
-    broadcastable to [B, N, Sq, Sk] with 1 = may attend."""
+    broadcastable to [B, N, Sq, Sk] with 1 = may attend.  ``bias`` is a float
+    array broadcastable to [B, N, Sq, Sk] added to the scores (a dense pse or
+    a float atten_mask; -inf entries mask their pair)."""
     if layout == "BSH" and n_heads is None:
         raise ValueError("BSH layout needs n_heads")
     q, k, v, B, N, Sq, Sk, D = _prep(q, k, v, n_heads, layout)
     mh = _MaskHolder(B, N, Sq, Sk, causal, kv_len, mask, modality_ids, allow,
-                     allow_diag)
+                     allow_diag, bias)
     sl = None
     if slopes is not None:
         sl = np.ascontiguousarray(_f64(slopes).reshape(N))
@@ -232,14 +245,14 @@ def fwd(q, k, v, scale, *, n_heads=None, layout="BNSD", causal=False,
 
 def bwd(q, k, v, dout, scale, *, n_heads=None, layout="BNSD", causal=False,
         kv_len=None, mask=None, modality_ids=None, allow=((1, 1), (0, 1)),
-        allow_diag=False, slopes=None):
+        allow_diag=False, slopes=None, bias=None):
     """Gradients (dq, dk, dv) of sum(dout * out) in fp64, layouts as the inputs."""
     if layout == "BSH" and n_heads is None:
         raise ValueError("BSH layout needs n_heads")
     q, k, v, B, N, Sq, Sk, D = _prep(q, k, v, n_heads, layout)
     do = _to_bnsd(_f64(dout), layout, n_heads)
     mh = _MaskHolder(B, N, Sq, Sk, causal, kv_len, mask, modality_ids, allow,
-                     allow_diag)
+                     allow_diag, bias)
     sl = None
     if slopes is not None:
         sl = np.ascontiguousarray(_f64(slopes).reshape(N))
@@ -258,14 +271,14 @@ def bwd(q, k, v, dout, scale, *, n_heads=None, layout="BNSD", causal=False,
 
 def probs(q, k, scale, b, h, *, n_heads=None, layout="BNSD", causal=False,
           kv_len=None, mask=None, modality_ids=None, allow=((1, 1), (0, 1)),
-          allow_diag=False, slopes=None):
+          allow_diag=False, slopes=None, bias=None):
     """Explicit probability matrix P [Sq, Sk] and lse [Sq] of one (b, h)."""
     q = _to_bnsd(_f64(q), layout, n_heads)
     k = _to_bnsd(_f64(k), layout, n_heads)
     B, N, Sq, D = q.shape
     Sk = k.shape[2]
     mh = _MaskHolder(B, N, Sq, Sk, causal, kv_len, mask, modality_ids, allow,
-                     allow_diag)
+                     allow_diag, bias)
     sl = None
     if slopes is not None:
         sl = np.ascontiguousarray(_f64(slopes).reshape(N))

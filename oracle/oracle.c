@@ -8,12 +8,17 @@
  *
  * What it computes (per batch b, head h, query row i, key j):
  *
- *   s_ij = scale * sum_d Q_id K_jd + bias_h(i, j)
+ *   s_ij = scale * sum_d Q_id K_jd + bias_h(i, j) + A[b,h,i,j]
  *          -- "FlashAttentionScore fusion operator replacement guide", sec. 2
  *             (the attention formula) and sec. 4 step 1 (matmul * scale,
  *             then the additive mask, softmax, matmul with V).
  *   bias_h(i, j) = -slope_h * |i - j|   (ALiBi position bias, the optional
  *             `pse` input of sec. 3.2 of the same guide), or 0 without pse.
+ *   A[b,h,i,j] = a dense additive term (the general `pse` tensor of sec. 3.2,
+ *             or a float `atten_mask` added to the scores as in sec. 4 step
+ *             1), broadcast over b and h by zero strides, or 0 without one.
+ *             Its values are finite or -inf; an s_ij of -inf counts as a
+ *             disallowed pair below (the same as masked_fill with -inf).
  *   allowed(i, j) = AND of the active rules
  *        causal   : j <= i             (lower-triangular `tril` mask,
  *                                       CogVLM page, "attention mask mechanism")
@@ -62,6 +67,9 @@ typedef struct {
   int64_t msb, msh, msq;
   const int32_t* ids;      /* [B][S] modality ids (0/1) or NULL; Sq == Sk */
   int allow00, allow01, allow10, allow11, allow_diag;
+  const double* add;       /* dense additive term or NULL; element (b,h,i,j)
+                              at b*asb + h*ash + i*asq + j */
+  int64_t asb, ash, asq;
 } oracle_mask;
 
 static int oracle_threads = 0;
@@ -118,6 +126,11 @@ static void probs_one_head(int b, int h, int Sq, int Sk, int D,
         dot += q[(int64_t)i * D + d] * k[(int64_t)j * D + d];
       double val = scale * dot;
       if (slopes) val += -slopes[h] * fabs((double)(i - j));
+      if (m && m->add) val += m->add[b * m->asb + h * m->ash + (int64_t)i * m->asq + j];
+      if (val == -INFINITY) { /* an additive -inf masks the pair */
+        *sij = -INFINITY;
+        continue;
+      }
       *sij = val;
       if (!any || val > mx) mx = val;
       any = 1;

@@ -31,6 +31,14 @@ MUTATIONS = {
                          "if (m->allow_diag && i == j) ok = ok;"),
     "diagonal_on_ids": ("if (m->allow_diag && i == j) ok = 1;",
                         "if (m->allow_diag && a == c) ok = 1;"),
+    "additive_ignored": ("if (m && m->add) val += m->add[b * m->asb + h * m->ash + (int64_t)i * m->asq + j];",
+                         "if (m && m->add) val += 0.0;"),
+    "additive_transposed": ("if (m && m->add) val += m->add[b * m->asb + h * m->ash + (int64_t)i * m->asq + j];",
+                            "if (m && m->add) val += m->add[b * m->asb + h * m->ash + (int64_t)(j % Sq) * m->asq + (i % Sk)];"),
+    "additive_sign": ("if (m && m->add) val += m->add[b * m->asb + h * m->ash + (int64_t)i * m->asq + j];",
+                      "if (m && m->add) val -= m->add[b * m->asb + h * m->ash + (int64_t)i * m->asq + j];"),
+    "additive_neginf_kept": ("      if (val == -INFINITY) { /* an additive -inf masks the pair */",
+                             "      if (0) { /* an additive -inf masks the pair */"),
     "dq_uses_q": ("acc += ds[(int64_t)i * Sk + j] * kh[(int64_t)j * D + d];",
                   "acc += ds[(int64_t)i * Sk + j] * qh[(int64_t)j * D + d];"),
 }
@@ -46,6 +54,9 @@ CHECKS = [
     lambda: pins.test_matches_torch_sdpa_fwd_bwd("causal", (13, 13)),
     lambda: pins.test_matches_torch_sdpa_fwd_bwd("padding", (7, 19)),
     lambda: pins.test_bwd_finite_differences("none", True),
+    lambda: pins.test_bias_of_zero_and_neginf_equals_the_bool_mask("bool"),
+    lambda: pins.test_bias_constant_shift_moves_only_the_lse((2, 3, 6, 9)),
+    pins.test_bias_q0_closed_form,
 ]
 
 

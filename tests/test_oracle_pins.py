@@ -408,3 +408,131 @@ def test_bwd_closed_form_invariants(mode):
     kw.pop("slopes")
     _, dk0, _ = oracle.bwd(np.zeros_like(q), k, v, do, 0.7, **kw)
     assert np.all(dk0 == 0.0)
+
+
+# ---------------------------------------------------------------- dense additive term
+# The general `pse` tensor and the float `atten_mask` of the FlashAttentionScore
+# guide (sec. 3.2; sec. 4 step 1 adds the mask to the scaled scores before the
+# softmax).  Pinned to the bool-mask path, to a shift invariance, to
+# torch's scaled_dot_product_attention with a float attn_mask, to scipy's
+# softmax for Q = 0, and to finite differences.
+
+def _bias(shape, seed, scale=2.0):
+    return _rand(shape, seed) * scale
+
+
+@pytest.mark.parametrize("mode", ["none", "causal", "padding", "bool"])
+def test_bias_of_zero_and_neginf_equals_the_bool_mask(mode):
+    B, N, Sq, Sk, D = 2, 3, 7, 11, 5
+    if mode == "causal":
+        Sk = Sq
+    q, k, v, do = (_rand(s, 90 + n) for n, s in enumerate(
+        [(B, N, Sq, D), (B, N, Sk, D), (B, N, Sk, D), (B, N, Sq, D)]))
+    kw = _mask_kwargs(mode, B, N, Sq, Sk, seed=95)
+    rng = np.random.default_rng(96)
+    keep = rng.random((B, N, Sq, Sk)) < 0.55
+    keep[0, 1, 2, :] = False            # one row with no key at all
+    add = np.where(keep, 0.0, -np.inf)
+    base = kw.pop("mask", None)        # "bool": the additive term on top of a bool mask
+    both = keep if base is None else (keep & (base != 0))
+    kw2 = dict(kw) if base is None else dict(kw, mask=base)
+    o1, l1 = oracle.fwd(q, k, v, 0.45, mask=both.astype(np.uint8), **kw)
+    o2, l2 = oracle.fwd(q, k, v, 0.45, bias=add, **kw2)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    assert l2[0, 1, 2] == -np.inf and np.all(o2[0, 1, 2] == 0.0)
+    g1 = oracle.bwd(q, k, v, do, 0.45, mask=both.astype(np.uint8), **kw)
+    g2 = oracle.bwd(q, k, v, do, 0.45, bias=add, **kw2)
+    for a, b in zip(g1, g2):
+        np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("shape", [(2, 3, 6, 9), (1, 3, 6, 9), (2, 1, 6, 9), (6, 9)])
+def test_bias_constant_shift_moves_only_the_lse(shape):
+    B, N, Sq, Sk, D = 2, 3, 6, 9, 4
+    q, k, v, do = (_rand(s, 100 + n) for n, s in enumerate(
+        [(B, N, Sq, D), (B, N, Sk, D), (B, N, Sk, D), (B, N, Sq, D)]))
+    add = _bias(shape, 105)
+    c = 3.25
+    kw = dict(slopes=np.array([0.2, 0.5, 0.05]), kv_len=np.array([9, 4], dtype=np.int32))
+    o1, l1 = oracle.fwd(q, k, v, 0.6, bias=add, **kw)
+    o2, l2 = oracle.fwd(q, k, v, 0.6, bias=add + c, **kw)
+    np.testing.assert_allclose(o2, o1, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(l2, l1 + c, atol=1e-12, rtol=0)
+    for a, b in zip(oracle.bwd(q, k, v, do, 0.6, bias=add, **kw),
+                    oracle.bwd(q, k, v, do, 0.6, bias=add + c, **kw)):
+        np.testing.assert_allclose(b, a, atol=1e-12, rtol=0)
+    # and a broadcast bias equals its materialised copy
+    full = np.broadcast_to(add.reshape((1,) * (4 - add.ndim) + add.shape), (B, N, Sq, Sk))
+    o3, l3 = oracle.fwd(q, k, v, 0.6, bias=full.copy(), **kw)
+    np.testing.assert_array_equal(o3, o1)
+    np.testing.assert_array_equal(l3, l1)
+
+
+@pytest.mark.parametrize("mode", ["none", "causal", "padding"])
+@pytest.mark.parametrize("sq_sk", [(9, 9), (5, 14)])
+def test_bias_matches_torch_sdpa_float_mask(mode, sq_sk):
+    Sq, Sk = sq_sk
+    if mode == "causal" and Sq != Sk:
+        pytest.skip("square causal case only")
+    B, N, D = 2, 2, 6
+    scale = 0.41
+    gen = torch.Generator().manual_seed(110)
+    q, do = (torch.randn(B, N, Sq, D, dtype=torch.float64, generator=gen) for _ in range(2))
+    k, v = (torch.randn(B, N, Sk, D, dtype=torch.float64, generator=gen) for _ in range(2))
+    add = torch.randn(1, N, Sq, Sk, dtype=torch.float64, generator=gen) * 1.5
+    kw = _mask_kwargs(mode, B, N, Sq, Sk, seed=111)
+    allowed = _allowed_dense(mode, B, N, Sq, Sk, kw)
+    nonempty = allowed.any(-1)
+    am = add.expand(B, N, Sq, Sk).masked_fill(~allowed, float("-inf"))
+    am = am.masked_fill(~nonempty[..., None], 0.0)   # torch gives NaN on empty rows
+    qt, kt, vt = (t.clone().requires_grad_(True) for t in (q, k, v))
+    ref = F.scaled_dot_product_attention(qt, kt, vt, attn_mask=am, scale=scale)
+    (ref * do * nonempty[..., None]).sum().backward()
+    out, lse = oracle.fwd(q, k, v, scale, bias=add.numpy(), **kw)
+    ne = nonempty.numpy()
+    np.testing.assert_allclose(out[ne], ref.detach().numpy()[ne], atol=1e-12, rtol=0)
+    s = (q @ k.transpose(-1, -2)) * scale + add
+    ref_lse = torch.logsumexp(s.masked_fill(~allowed, float("-inf")), -1).numpy()
+    np.testing.assert_allclose(lse[ne], ref_lse[ne], atol=1e-12, rtol=0)
+    dq, dk, dv = oracle.bwd(q, k, v, do * nonempty[..., None], scale, bias=add.numpy(), **kw)
+    np.testing.assert_allclose(dq, qt.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), atol=1e-12, rtol=0)
+
+
+def test_bias_q0_closed_form():
+    from scipy.special import logsumexp, softmax
+    B, N, Sq, Sk, D = 2, 2, 5, 8, 3
+    q = np.zeros((B, N, Sq, D))
+    k = _rand((B, N, Sk, D), 120)
+    v = _rand((B, N, Sk, D), 121)
+    add = _bias((B, N, Sq, Sk), 122, scale=3.0)   # not symmetric in (i, j)
+    add[1, 0, 3, 5:] = -np.inf
+    out, lse = oracle.fwd(q, k, v, 0.9, bias=add)
+    np.testing.assert_allclose(lse, logsumexp(add, axis=-1), atol=1e-13, rtol=0)
+    want = np.einsum("bnij,bnjd->bnid", softmax(add, axis=-1), v)
+    np.testing.assert_allclose(out, want, atol=1e-13, rtol=0)
+
+
+@pytest.mark.parametrize("mode", ["none", "causal"])
+def test_bias_bwd_finite_differences(mode):
+    B, N, S, D = 1, 2, 5, 3
+    q, k, v, do = (_rand((B, N, S, D), 130 + n) for n in range(4))
+    kw = _mask_kwargs(mode, B, N, S, S, seed=134)
+    kw["bias"] = _bias((1, N, S, S), 135)
+    dq, dk, dv = oracle.bwd(q, k, v, do, 0.8, **kw)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            args = {"q": q, "k": k, "v": v}
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args[name] = xp
+            lp = _loss(args["q"], args["k"], args["v"], do, 0.8, kw)
+            args[name] = xm
+            lm = _loss(args["q"], args["k"], args["v"], do, 0.8, kw)
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.abs(fd - g).max() / max(1.0, np.abs(g).max())
+        assert err < 1e-6, (name, err)
