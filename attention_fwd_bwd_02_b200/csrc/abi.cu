@@ -111,11 +111,21 @@ fa_status make_problem(const fa_shape* s, const fa_pse* pse, const fa_mask* m,
     }
   }
   if (pse) {
-    if (pse->kind == FA_PSE_ALIBI) {
+    if (pse->kind & ~(FA_PSE_ALIBI | FA_PSE_DENSE)) return FA_ERR_INVALID_ARG;
+    if (pse->kind & FA_PSE_ALIBI) {
       if (!pse->slopes) return FA_ERR_INVALID_ARG;
       q.slopes = pse->slopes;
-    } else if (pse->kind != FA_PSE_NONE) {
-      return FA_ERR_INVALID_ARG;
+    }
+    if (pse->kind & FA_PSE_DENSE) {
+      if (!pse->bias || (reinterpret_cast<uintptr_t>(pse->bias) & 3u)) return FA_ERR_INVALID_ARG;
+      if (pse->bias_stride_b < 0 || pse->bias_stride_h < 0 || pse->bias_stride_q < s->Sk)
+        return FA_ERR_INVALID_ARG;
+      q.add = pse->bias;
+      q.a_sb = pse->bias_stride_b;
+      q.a_sh = pse->bias_stride_h;
+      q.a_sq = pse->bias_stride_q;
+      q.add_vec = aligned16(pse->bias) && pse->bias_stride_b % 4 == 0 &&
+                  pse->bias_stride_h % 4 == 0 && pse->bias_stride_q % 4 == 0;
     }
   }
   *p = q;

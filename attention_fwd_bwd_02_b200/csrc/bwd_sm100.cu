@@ -146,7 +146,9 @@ __device__ __forceinline__ int count_qtiles(const Problem& p, const KeyCtx& c) {
 __device__ __forceinline__ int col0_dq(int D, int wq) { return wq * (D / 4); }
 
 // kF16 selects fp16 operands (Q, K, V, dO, P, dS, dK, dV); bf16 otherwise.
-template <int D, bool kF16>
+// kAdd: the problem has a dense additive term (p.add); a kernel of its own so
+// that the other kernels keep its registers.
+template <int D, bool kF16, bool kAdd>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_sm100(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_k,
@@ -177,8 +179,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = tid & 31;
 
   KeyCtx c;
-  c.b = blockIdx.z;
-  c.h = blockIdx.y;
+  // A dense term shared by the batches: the grid runs the batches of one
+  // head together (y = batch, z = head), so its tiles come from L2.
+  const bool b_major = p.add && p.a_sb == 0;
+  c.b = b_major ? blockIdx.y : blockIdx.z;
+  c.h = b_major ? blockIdx.z : blockIdx.y;
   c.k0 = blockIdx.x * kBN;
   c.k_last = min(c.k0 + kBN, p.Sk) - 1;
   c.nkeys = visible_keys(p, c.b);
@@ -377,6 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has_alibi = p.slopes != nullptr;
     const bool causal = p.mask_flags & FA_MASK_CAUSAL;
     const bool fold = has_alibi && causal;  // ALiBi linear in i - j
+    constexpr bool has_add = kAdd;           // dense additive term (p.add)
     const float abs_g = fold ? 0.f : -slope_l2;  // |i - j| form otherwise
     const int32_t* ids = (p.mask_flags & FA_MASK_MODALITY) ? p.ids + int64_t(c.b) * p.Sk : nullptr;
     const int id_j = (ids && j < p.Sk) ? (ids[j] & 1) : 0;
@@ -404,9 +410,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int i = q0 + 32 * u + lane;
+        // A row with no visible pair (LSE = -inf) stages -inf, so that every
+        // x of the row is -inf and P = 0 there.
+        const float lse_i = i < p.Sq ? lse[row_base + i] : -INFINITY;
         st_shared_f32(st_w + 4 * (32 * u + lane),
-                      i < p.Sq ? fmaf(col_g, float(32 * u + lane), -lse[row_base + i] * kLog2e)
-                               : -INFINITY);
+                      lse_i != -INFINITY ? fmaf(col_g, float(32 * u + lane), -lse_i * kLog2e)
+                                         : -INFINITY);
         st_shared_f32(st_w + 4 * (kBM + 32 * u + lane), i < p.Sq ? -delta[row_base + i] : 0.f);
       }
       __syncwarp();
@@ -438,6 +447,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
+      // The dense additive term A[i][j] of the 64 queries for key j (0
+      // outside the arrays, where the pair is masked), 32 queries at a
+      // time; the first 32 are requested before S is ready.
+      const bool a_in = has_add && j < p.Sk;
+      const float* acol = has_add ? p.add + c.b * p.a_sb + c.h * p.a_sh + (a_in ? j : 0) : nullptr;
+      float av[32];
+      if (has_add) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          av[e] = (a_in && q0 + e < p.Sq) ? __ldg(acol + int64_t(q0 + e) * p.a_sq) : 0.f;
+      }
       const bool got_s = mbar_wait_s(BAR(C::bSFull + b), mine & 1, abort_addr);
       if (!__all_sync(~0u, got_s)) { ok = false; return false; }
       tc_fence_after();
@@ -459,9 +479,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint64_t brow2 = f2_pack(brow, brow);
 #pragma unroll
         for (int e = 0; e < kBM; e += 2) {
+          if (has_add && e == 32) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+              av[u] = (a_in && q0 + 32 + u < p.Sq) ? __ldg(acol + int64_t(q0 + 32 + u) * p.a_sq) : 0.f;
+          }
           const float2 nl = ld_shared_f2(st + 4 * e);
           uint64_t off2 = f2_pack(nl.x, nl.y);
           if (fold) off2 = fadd2(off2, brow2);
+          if (has_add)
+            off2 = ffma2(f2_pack(av[e & 31], av[(e & 31) + 1]), f2_pack(kLog2e, kLog2e), off2);
           float x0, x1;
           f2_unpack(ffma2(f2_pack(__uint_as_float(sr[e >> 5][e & 31]),
                                   __uint_as_float(sr[e >> 5][(e & 31) + 1])),
@@ -572,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0 && ld_shared_volatile(abort_addr)) atomicOr(p.status, 1u);
 }
 
-template <int D, bool kF16>
+template <int D, bool kF16, bool kAdd>
 cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
                          const void* v, const void* dout, const float* lse,
                          const float* delta, float* dq_acc, void* dk, void* dv,
@@ -593,12 +620,12 @@ cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
   // the increase waiting.
   static std::atomic<uint64_t> ready{0};
   e = once_per_device(ready, []() -> cudaError_t {
-    cudaError_t r = cudaFuncSetAttribute(bwd_sm100<D, kF16>,
+    cudaError_t r = cudaFuncSetAttribute(bwd_sm100<D, kF16, kAdd>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (r != cudaSuccess) return r;
     cudaFuncAttributes fa_attr;
-    if ((r = cudaFuncGetAttributes(&fa_attr, bwd_sm100<D, kF16>)) != cudaSuccess) return r;
+    if ((r = cudaFuncGetAttributes(&fa_attr, bwd_sm100<D, kF16, kAdd>)) != cudaSuccess) return r;
     return fa_attr.numRegs * kThreads <
                    2 * 128 * int(kRegsSoftmax) + 128 * int(kRegsDq) + 128 * int(kRegsControl)
                ? cudaErrorInvalidConfiguration
@@ -606,7 +633,8 @@ cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
   });
   if (e != cudaSuccess) return e;
   dim3 grid((p.Sk + kBN - 1) / kBN, p.N, p.B);
-  bwd_sm100<D, kF16><<<grid, kThreads, C::kSmemBytes, st>>>(
+  if (p.add && p.a_sb == 0) grid = dim3((p.Sk + kBN - 1) / kBN, p.B, p.N);
+  bwd_sm100<D, kF16, kAdd><<<grid, kThreads, C::kSmemBytes, st>>>(
       tq, tk, tv, tdo, tdq, p, lse, delta, static_cast<uint16_t*>(dk),
       static_cast<uint16_t*>(dv));
   return cudaGetLastError();
@@ -618,12 +646,18 @@ cudaError_t launch_bwd_sm100(const Problem& p, const void* q, const void* k,
                              const void* v, const void* dout, const float* lse,
                              const float* delta, float* dq_acc, void* dk, void* dv,
                              cudaStream_t st) {
-  if (p.D == 64)
-    return p.f16 ? launch_bwd_d<64, true>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st)
-                 : launch_bwd_d<64, false>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
-  if (p.D == 128)
-    return p.f16 ? launch_bwd_d<128, true>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st)
-                 : launch_bwd_d<128, false>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
+#define FA_BWD_CASE(HD, F16, ADD) \
+  if (p.D == HD && bool(p.f16) == F16 && (p.add != nullptr) == ADD) \
+    return launch_bwd_d<HD, F16, ADD>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
+  FA_BWD_CASE(64, false, false)
+  FA_BWD_CASE(64, true, false)
+  FA_BWD_CASE(128, false, false)
+  FA_BWD_CASE(128, true, false)
+  FA_BWD_CASE(64, false, true)
+  FA_BWD_CASE(64, true, true)
+  FA_BWD_CASE(128, false, true)
+  FA_BWD_CASE(128, true, true)
+#undef FA_BWD_CASE
   return cudaErrorInvalidValue;
 }
 

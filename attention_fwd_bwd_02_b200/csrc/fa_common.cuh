@@ -27,6 +27,9 @@ struct Problem {
   const int32_t* ids;       // modality ids [B][Sk]
   uint32_t allow_bits;      // bit (2*id_q + id_k): allowed; bit 4: diagonal
   const float* slopes;      // ALiBi slopes [N] or null
+  const float* add;         // dense additive term (pse tensor / float mask) or null
+  int64_t a_sb, a_sh, a_sq; // its strides in elements (0 = broadcast)
+  uint32_t add_vec;         // 1: 16-byte aligned rows, float4 loads allowed
   uint32_t f16;             // tensor-core path: 1 = fp16 operands, 0 = bf16
   uint32_t debug_flags;     // test hooks, 0 in production (kDebug* below)
   unsigned int* status;     // device status word (bit 0: a wait timed out)
@@ -98,6 +101,11 @@ __device__ __forceinline__ uint32_t modality_row_bits(uint32_t allow_bits,
 }
 
 // ALiBi bias of (h, i, j) in natural units: -slope_h * |i - j|.
+// Dense additive term A[b][h][i][j] (pse tensor / float mask), i < Sq, j < Sk.
+__device__ __forceinline__ float add_term(const Problem& p, int b, int h, int i, int j) {
+  return p.add[b * p.a_sb + h * p.a_sh + int64_t(i) * p.a_sq + j];
+}
+
 __device__ __forceinline__ float alibi_bias(const Problem& p, int h, int i,
                                             int j) {
   int d = i - j;

@@ -160,6 +160,30 @@ __device__ __forceinline__ int kt_at(const Item& c, int it) {
   return it <= c.kt_pivot ? c.kt_pivot - it : it;
 }
 
+// Keys 32*q4 .. 32*q4+31 of one row of the dense additive term (row pointer
+// at the tile's first key; `lim` keys of the tile exist), as 8 float4.
+// Absent keys read 0 (they are masked by the tile classification).
+__device__ __forceinline__ void load_add_chunk(const float* arow, bool vec, int q4, int lim,
+                                               float4 (&a)[8]) {
+  if (!arow) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+  } else if (vec) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a[u] = __ldg(reinterpret_cast<const float4*>(arow + 32 * q4) + u);
+  } else {
+    float v[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) v[e] = (32 * q4 + e < lim) ? __ldg(arow + 32 * q4 + e) : 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a[u] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+  }
+}
+
+__device__ __forceinline__ float f4_get(const float4& a, int k) {
+  return k == 0 ? a.x : (k == 1 ? a.y : (k == 2 ? a.z : a.w));
+}
+
 // Work item number idx of the claim order.  Heads are taken in groups of
 // `group` heads (sized so that their K and V stay in L2 together); within a
 // group, query blocks go longest first under the causal mask (all heads'
@@ -176,8 +200,15 @@ __device__ __forceinline__ Item make_item(const Problem& p, int idx, int q_block
   const int band = r / g_heads;
   const int bh = g * group + (r - band * g_heads);
   const int qb = causal ? (q_blocks - 1 - band) : band;
-  c.b = bh / p.N;
-  c.h = bh - c.b * p.N;
+  if (p.add && p.a_sb == 0) {
+    // A dense term shared by the batches: the batches of one head run
+    // together, so that its tiles are read from L2 after the first.
+    c.h = bh / p.B;
+    c.b = bh - c.h * p.B;
+  } else {
+    c.b = bh / p.N;
+    c.h = bh - c.b * p.N;
+  }
   c.nkeys = visible_keys(p, c.b);
   c.kt_end = 0;
 #pragma unroll
@@ -267,8 +298,9 @@ __device__ __forceinline__ int tile_class(const Problem& p, const Item& c, int t
   return cls;
 }
 
-// kF16 selects fp16 operands (Q, K, V, P, out); bf16 otherwise.
-template <int D, bool kF16>
+// kF16 selects fp16 operands (Q, K, V, P, out); bf16 otherwise.  kAdd: the
+// problem has a dense additive term (p.add), in a kernel of its own.
+template <int D, bool kF16, bool kAdd>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_k,
@@ -565,6 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + C::kColO + t * D;
     const float sl2 = p.scale_log2;
     const bool has_alibi = p.slopes != nullptr;
+    constexpr bool has_add = kAdd;
     int steps = 0, o_uses = 0;
     bool ok = true;
 
@@ -603,23 +636,63 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t kid = key_tile_ids(p, c, kt);
         const int cls = tile_class(p, c, t, kt, kid);
         if (cls == 0) continue;
+        const int k0 = kt * kBN;
+        // The dense additive term of this row: the next tile's row is
+        // brought into L2 while this one is processed.
+        const float* arow = (has_add && row_real)
+                                ? p.add + c.b * p.a_sb + c.h * p.a_sh + int64_t(i) * p.a_sq + k0
+                                : nullptr;
+        const bool a_vec = p.add_vec && k0 + kBN <= p.Sk;
+        if (has_add) {
+          if (row_real && it + 1 < c.kt_end) {
+            const int k1 = kt_at(c, it + 1) * kBN;
+            const float* an = p.add + c.b * p.a_sb + c.h * p.a_sh + int64_t(i) * p.a_sq + k1;
+#pragma unroll
+            for (int m4 = 0; m4 < 4; ++m4)
+              if (k1 + 32 * m4 < p.Sk) prefetch_l2(an + 32 * m4);
+          }
+        }
         // Every wait is agreed warp-wide before the .sync.aligned TMEM ops.
         const bool got_s = mbar_wait_s(BAR(C::bSFull + t), steps & 1, abort_addr);
         if (!__all_sync(~0u, got_s)) { ok = false; break; }
         tc_fence_after();
-        const int k0 = kt * kBN;
         // Without a bias and with a positive scale, max(s * c) = c * max(s)
         // exactly, and x - m folds into one fma per element; the same
         // arithmetic is used whether or not the tile needs masking, so the
         // result does not depend on the tile classification.
-        const bool plain = !has_alibi && sl2 > 0.f;
+        const bool plain = !has_alibi && !has_add && sl2 > 0.f;
         const bool masked = cls == 1;
+        if (has_add) {
+          // x = s * scale * log2(e) + log2(e) * (A + ALiBi), 32 keys at a
+          // time, written back over S; the term's next 32 keys load while
+          // these are processed.
+          float4 a_nx[8];
+          load_add_chunk(arow, a_vec, 0, p.Sk - k0, a_nx);
+#pragma unroll 1
+          for (int q4 = 0; q4 < 4; ++q4) {
+            float4 a_cu[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) a_cu[u] = a_nx[u];
+            if (q4 < 3) load_add_chunk(arow, a_vec, q4 + 1, p.Sk - k0, a_nx);
+            uint32_t s32[32];
+            tmem_ld32(tS + q4 * 32, s32);
+            tmem_ld_wait(s32);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              float b = f4_get(a_cu[e >> 2], e & 3);
+              if (has_alibi) b = fmaf(-slope_l2 * kLn2, fabsf(float(k0 + 32 * q4 + e - i)), b);
+              s32[e] = __float_as_uint(fmaf(__uint_as_float(s32[e]), sl2, b * kLog2e));
+            }
+            tmem_st32(tS + q4 * 32, s32);
+          }
+          tmem_st_wait();
+        }
         uint32_t sr[4][32];
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) tmem_ld32(tS + q4 * 32, sr[q4]);
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) tmem_ld_wait(sr[q4]);
-        if (!plain) {
+        if (!plain && !has_add) {
           // x = s * scale * log2(e) + ALiBi, kept in sr.  The bias
           // -slope * log2(e) * |i - j| is linear in the key column e when
           // the tile lies on one side of the diagonal, and under the causal
@@ -821,7 +894,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <int D, bool kF16>
+template <int D, bool kF16, bool kAdd>
 static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
                                 const void* v, void* out, float* lse,
                                 cudaStream_t st) {
@@ -836,12 +909,12 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   // with fewer registers per thread would leave the increase waiting.
   static std::atomic<uint64_t> ready{0};
   e = once_per_device(ready, []() -> cudaError_t {
-    cudaError_t r = cudaFuncSetAttribute(fwd_sm100<D, kF16>,
+    cudaError_t r = cudaFuncSetAttribute(fwd_sm100<D, kF16, kAdd>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (r != cudaSuccess) return r;
     cudaFuncAttributes fa_attr;
-    if ((r = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16>)) != cudaSuccess) return r;
+    if ((r = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16, kAdd>)) != cudaSuccess) return r;
     return fa_attr.numRegs < int(kRegsLaunch) ? cudaErrorInvalidConfiguration : cudaSuccess;
   });
   if (e != cudaSuccess) return e;
@@ -857,7 +930,7 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   group = group < 1 ? 1 : (group > p.B * p.N ? p.B * p.N : group);
   unsigned int* ctr = work_counter();
   if (!ctr) return cudaErrorUnknown;
-  fwd_sm100<D, kF16><<<grid, kThreads, C::kSmemBytes, st>>>(
+  fwd_sm100<D, kF16, kAdd><<<grid, kThreads, C::kSmemBytes, st>>>(
       tq, tk, tv, p, static_cast<uint16_t*>(out), lse, q_blocks, int(items), group, ctr);
   return cudaGetLastError();
 }
@@ -865,12 +938,18 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
 cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k,
                              const void* v, void* out, float* lse,
                              cudaStream_t st) {
-  if (p.D == 64)
-    return p.f16 ? launch_fwd_d<64, true>(p, q, k, v, out, lse, st)
-                 : launch_fwd_d<64, false>(p, q, k, v, out, lse, st);
-  if (p.D == 128)
-    return p.f16 ? launch_fwd_d<128, true>(p, q, k, v, out, lse, st)
-                 : launch_fwd_d<128, false>(p, q, k, v, out, lse, st);
+#define FA_FWD_CASE(HD, F16, ADD) \
+  if (p.D == HD && bool(p.f16) == F16 && (p.add != nullptr) == ADD) \
+    return launch_fwd_d<HD, F16, ADD>(p, q, k, v, out, lse, st);
+  FA_FWD_CASE(64, false, false)
+  FA_FWD_CASE(64, true, false)
+  FA_FWD_CASE(128, false, false)
+  FA_FWD_CASE(128, true, false)
+  FA_FWD_CASE(64, false, true)
+  FA_FWD_CASE(64, true, true)
+  FA_FWD_CASE(128, false, true)
+  FA_FWD_CASE(128, true, true)
+#undef FA_FWD_CASE
   return cudaErrorInvalidValue;
 }
 

@@ -87,6 +87,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
         for (int d = 0; d < D; ++d) dot = fmaf(sQ[rl][d], sK[lane][d], dot);
         s = dot * p.scale;
         if (p.slopes) s += alibi_bias(p, h, i, j);
+        if (p.add) s += add_term(p, b, h, i, j);
       }
       float tmax = s;
 #pragma unroll
@@ -200,6 +201,7 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         }
         float s = dot * p.scale;
         if (p.slopes) s += alibi_bias(p, h, i, j);
+        if (p.add) s += add_term(p, b, h, i, j);
         pj = expf(s - lse_i);
         dsj = pj * (dpd - dl_i);
       }

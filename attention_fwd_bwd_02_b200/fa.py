@@ -30,7 +30,7 @@ TESTING_HEADER = os.path.join(os.path.dirname(_HERE), "include", "fa_testing.h")
 FA_LAYOUT_BNSD, FA_LAYOUT_BSH = 0, 1
 FA_F32, FA_BF16, FA_F16 = 0, 1, 2
 FA_MASK_CAUSAL, FA_MASK_KV_PADDING, FA_MASK_BOOL, FA_MASK_MODALITY = 1, 2, 4, 8
-FA_PSE_NONE, FA_PSE_ALIBI = 0, 1
+FA_PSE_NONE, FA_PSE_ALIBI, FA_PSE_DENSE = 0, 1, 2
 FA_TILE_M = FA_TILE_N = 128
 
 
@@ -61,7 +61,9 @@ class FaMask(ctypes.Structure):
 
 
 class FaPse(ctypes.Structure):
-    _fields_ = [("kind", ctypes.c_int), ("slopes", ctypes.c_void_p)]
+    _fields_ = [("kind", ctypes.c_int), ("slopes", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("bias_stride_b", ctypes.c_int64),
+                ("bias_stride_h", ctypes.c_int64), ("bias_stride_q", ctypes.c_int64)]
 
 
 _lib = None
@@ -190,6 +192,14 @@ def _check_operand(t, shape, name, like=None):
         raise FaError(FA_ERR_INVALID_ARG, f"{name} has shape {tuple(t.shape)}, want {tuple(shape)}")
 
 
+def _check_lse(lse, shape, like):
+    if lse is None or not lse.is_cuda or lse.dtype != torch.float32 or \
+            not lse.is_contiguous() or lse.device != like.device or \
+            tuple(lse.shape) != (shape.B, shape.N, shape.Sq):
+        raise FaError(FA_ERR_INVALID_ARG,
+                      f"lse must be a contiguous fp32 [B, N, Sq] tensor on q's device")
+
+
 class _Keep:
     """Holds tensors that a ctypes struct points to."""
 
@@ -242,12 +252,59 @@ def make_mask(shape: FaShape, *, causal=False, atten_mask=None, padding_kv_len=N
     return m if flags else None
 
 
-def make_pse(slopes: Optional[torch.Tensor], keep: _Keep) -> Optional[FaPse]:
-    if slopes is None:
-        return None
-    s = slopes.to(torch.float32).contiguous()
-    keep.items.append(s)
-    return FaPse(FA_PSE_ALIBI, s.data_ptr())
+def split_atten_mask(atten_mask):
+    """(bool mask, additive term): a bool/uint8 atten_mask selects pairs
+    (1 = may attend); a floating one is added to the scaled scores (the
+    guide's unfused steps, sec. 4 step 1)."""
+    if atten_mask is not None and atten_mask.is_floating_point():
+        return None, atten_mask
+    return atten_mask, None
+
+
+def _dense_term(t: torch.Tensor, shape: FaShape, keep: _Keep):
+    """Device fp32 view of a dense additive term broadcastable to
+    [B, N, Sq, Sk] (leading dims 1 or full); returns (ptr, sb, sh, sq)."""
+    if not t.is_cuda:
+        raise FaError(FA_ERR_INVALID_ARG, "the dense pse / float mask must be a CUDA tensor")
+    a = t if t.dtype == torch.float32 else t.to(torch.float32)
+    while a.dim() < 4:
+        a = a.unsqueeze(0)
+    if a.dim() != 4 or tuple(a.shape[-2:]) != (shape.Sq, shape.Sk) or \
+            a.shape[0] not in (1, shape.B) or a.shape[1] not in (1, shape.N):
+        raise FaError(FA_ERR_INVALID_ARG,
+                      f"dense pse / float mask of shape {tuple(t.shape)} does not broadcast "
+                      f"to [{shape.B}, {shape.N}, {shape.Sq}, {shape.Sk}]")
+    if a.stride(-1) != 1 or a.stride(-2) < shape.Sk or \
+            (a.shape[0] > 1 and a.stride(0) <= 0) or (a.shape[1] > 1 and a.stride(1) <= 0):
+        a = a.contiguous()
+    keep.items.append(a)
+    sb = 0 if a.shape[0] == 1 else a.stride(0)
+    sh = 0 if a.shape[1] == 1 else a.stride(1)
+    return a.data_ptr(), sb, sh, a.stride(2)
+
+
+def make_pse(pse: Optional[torch.Tensor], keep: _Keep, shape: Optional[FaShape] = None,
+             add: Optional[torch.Tensor] = None) -> Optional[FaPse]:
+    """pse: an ALiBi slope vector [N] or a dense term broadcastable to
+    [B, N, Sq, Sk]; add: a float atten_mask (another dense term).  Only one
+    dense term is taken."""
+    ps = FaPse()
+    if pse is not None and pse.dim() == 1:
+        s = pse.to(torch.float32).contiguous()
+        keep.items.append(s)
+        ps.kind |= FA_PSE_ALIBI
+        ps.slopes = s.data_ptr()
+    elif pse is not None:
+        if add is not None:
+            raise FaError(FA_ERR_UNSUPPORTED,
+                          "a dense pse and a float atten_mask: pass their sum as one of them")
+        add = pse
+    if add is not None:
+        if shape is None:
+            raise FaError(FA_ERR_INVALID_ARG, "a dense term needs the problem shape")
+        ps.bias, ps.bias_stride_b, ps.bias_stride_h, ps.bias_stride_q = _dense_term(add, shape, keep)
+        ps.kind |= FA_PSE_DENSE
+    return ps if ps.kind else None
 
 
 def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
@@ -257,8 +314,11 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
         _withhold_q=False) -> Tuple[torch.Tensor, torch.Tensor]:
     """Fused attention forward.  Returns (out, lse).
 
-    pse: ALiBi slope vector [N] (fp32) or None.  atten_mask: bool/uint8
-    tensor broadcastable to [B, N, Sq, Sk], 1 = may attend.  causal: the
+    pse: ALiBi slope vector [N] (fp32), a dense term broadcastable to
+    [B, N, Sq, Sk] added to the scaled scores, or None.  atten_mask:
+    bool/uint8 tensor broadcastable to [B, N, Sq, Sk], 1 = may attend, or a
+    floating tensor of that shape added to the scaled scores (finite or
+    -inf; -inf masks the pair).  causal: the
     lower-triangular rule.  padding_kv_len: int [B] valid keys per batch.
     modality_ids [B, S] with the 2x2 ``allow`` table and ``allow_diag``.
     scale has no default (pass 1/sqrt(D) explicitly)."""
@@ -269,15 +329,18 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
     _check_operand(key, None, "key", query)
     _check_operand(value, key.shape, "value", query)
     keep = _Keep()
+    atten_mask, add = split_atten_mask(atten_mask)
     m = make_mask(shape, causal=causal, atten_mask=atten_mask,
                   padding_kv_len=padding_kv_len, modality_ids=modality_ids,
                   allow=allow, allow_diag=allow_diag, tile_map=tile_map, keep=keep)
-    ps = make_pse(pse, keep)
+    ps = make_pse(pse, keep, shape, add)
     if out is None:
         out = torch.empty_like(query)
     if lse is None:
         lse = torch.empty((shape.B, shape.N, shape.Sq), dtype=torch.float32,
                           device=query.device)
+    _check_operand(out, query.shape, "out", query)
+    _check_lse(lse, shape, query)
     entry = lib().fa_testing_fwd_withhold_q if _withhold_q else lib().fa_fwd
     with _on_device(query.device):
         st = entry(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
@@ -314,16 +377,23 @@ def bwd(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
                  (dout, "dout")):
         _check_operand(t, None, n, query)
     keep = _Keep()
+    atten_mask, add = split_atten_mask(atten_mask)
     m = make_mask(shape, causal=causal, atten_mask=atten_mask,
                   padding_kv_len=padding_kv_len, modality_ids=modality_ids,
                   allow=allow, allow_diag=allow_diag, tile_map=tile_map, keep=keep)
-    ps = make_pse(pse, keep)
+    ps = make_pse(pse, keep, shape, add)
     need = bwd_workspace_size(shape)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=query.device)
     dq = torch.empty_like(query) if dq is None else dq
     dk = torch.empty_like(key) if dk is None else dk
     dv = torch.empty_like(value) if dv is None else dv
+    for t, like, n in ((dq, query, "dq"), (dk, key, "dk"), (dv, value, "dv")):
+        _check_operand(t, like.shape, n, query)
+    _check_lse(lse, shape, query)
+    if workspace.dtype != torch.uint8 or not workspace.is_contiguous() or \
+            workspace.device != query.device:
+        raise FaError(FA_ERR_INVALID_ARG, "workspace must be a contiguous uint8 tensor on q's device")
     with _on_device(query.device):
         st = lib().fa_bwd(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
                           _ptr(out), _ptr(dout), _ptr(lse),
@@ -354,13 +424,17 @@ def bwd_noalloc(query, key, value, out, dout, lse, head_num=None, input_layout="
                  (dout, "dout")):
         _check_operand(t, None, n, query)
     keep = _Keep()
+    atten_mask, add = split_atten_mask(atten_mask)
     m = make_mask(shape, causal=causal, atten_mask=atten_mask,
                   padding_kv_len=padding_kv_len, modality_ids=modality_ids,
                   allow=allow, allow_diag=allow_diag, tile_map=tile_map, keep=keep)
-    ps = make_pse(pse, keep)
+    ps = make_pse(pse, keep, shape, add)
     dq = torch.empty_like(query) if dq is None else dq
     dk = torch.empty_like(key) if dk is None else dk
     dv = torch.empty_like(value) if dv is None else dv
+    for t, like, n in ((dq, query, "dq"), (dk, key, "dk"), (dv, value, "dv")):
+        _check_operand(t, like.shape, n, query)
+    _check_lse(lse, shape, query)
     with _on_device(query.device):
         st = lib().fa_bwd_noalloc(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
                                   _ptr(out), _ptr(dout), _ptr(lse),

@@ -102,12 +102,26 @@ typedef struct {
 } fa_mask;
 
 /* Position bias `pse` (guide, sec. 3.2: "optional, supports fusing position
- * encodings such as ALiBi").  FA_PSE_ALIBI adds -slopes[h] * |i - j| to the
- * scaled score; the bias is not multiplied by `scale`. */
-enum { FA_PSE_NONE = 0, FA_PSE_ALIBI = 1 };
+ * encodings such as ALiBi").  `kind` is a bit set; each term is added to the
+ * scaled score and is not multiplied by `scale`:
+ *   FA_PSE_ALIBI adds -slopes[h] * |i - j|;
+ *   FA_PSE_DENSE adds a dense fp32 term A[b][h][i][j] -- the general pse
+ *     tensor of sec. 3.2, or a float attention mask added to the scaled
+ *     scores as in the guide's unfused steps (sec. 4 step 1).  Element
+ *     (b, h, i, j) is read at bias[b*bias_stride_b + h*bias_stride_h +
+ *     i*bias_stride_q + j] (strides in elements; 0 broadcasts over b or h,
+ *     and bias_stride_q >= Sk is required).  Values are finite or -inf: a
+ *     pair whose score is -inf is masked, and a row left with no finite
+ *     score gives out = 0, lse = -inf, as with the bool mask.  The array is
+ *     read, never written; 16-byte alignment of `bias` and strides that are
+ *     multiples of 4 take the vectorised loads (any 4-byte aligned array is
+ *     accepted).  FA_PSE_ALIBI | FA_PSE_DENSE adds both. */
+enum { FA_PSE_NONE = 0, FA_PSE_ALIBI = 1, FA_PSE_DENSE = 2 };
 typedef struct {
-  int kind;                     /* FA_PSE_*                                  */
+  int kind;                     /* FA_PSE_* bit set                          */
   const float* slopes;          /* [N] device, FA_PSE_ALIBI                  */
+  const float* bias;            /* device fp32, FA_PSE_DENSE                 */
+  int64_t bias_stride_b, bias_stride_h, bias_stride_q;
 } fa_pse;
 
 typedef struct {

@@ -100,7 +100,16 @@ def test_mask_validation(L):
 
 def test_pse_validation(L):
     assert _fwd(L, _shape(), pse=fa.FaPse(fa.FA_PSE_ALIBI, None)) == fa.FA_ERR_INVALID_ARG
-    assert _fwd(L, _shape(), pse=fa.FaPse(3, 0x10000)) == fa.FA_ERR_INVALID_ARG
+    assert _fwd(L, _shape(), pse=fa.FaPse(3, 0x10000)) == fa.FA_ERR_INVALID_ARG  # no dense array
+    assert _fwd(L, _shape(), pse=fa.FaPse(4, 0x10000)) == fa.FA_ERR_INVALID_ARG  # unknown kind
+    S = _shape()
+    ok = dict(bias=0x10000, bias_stride_b=0, bias_stride_h=0, bias_stride_q=S.Sk)
+    for bad in (dict(bias=0x10002), dict(bias_stride_q=S.Sk - 1), dict(bias_stride_b=-1),
+                dict(bias_stride_h=-4)):
+        kw = dict(ok, **bad)
+        ps = fa.FaPse(fa.FA_PSE_DENSE, None, kw["bias"], kw["bias_stride_b"],
+                      kw["bias_stride_h"], kw["bias_stride_q"])
+        assert _fwd(L, S, pse=ps) == fa.FA_ERR_INVALID_ARG, bad
 
 
 def test_empty_problems_are_ok_without_launch(L):
