@@ -57,6 +57,10 @@ class _Mask(ctypes.Structure):
         ("asb", ctypes.c_int64),
         ("ash", ctypes.c_int64),
         ("asq", ctypes.c_int64),
+        ("dropout", ctypes.c_int),
+        ("keep_prob", ctypes.c_double),
+        ("seed", ctypes.c_uint64),
+        ("offset", ctypes.c_uint64),
     ]
 
 
@@ -90,6 +94,10 @@ def _load():
         lib.oracle_probs.argtypes = [i, i, i, i, i, i, i, dp, dp, dp,
                                      ctypes.POINTER(_Mask), ctypes.c_double, dp, dp]
         lib.oracle_probs.restype = ctypes.c_int
+        lib.oracle_philox4x64.argtypes = [dp, dp, dp]
+        lib.oracle_philox4x64.restype = None
+        lib.oracle_dropout_mask.argtypes = [i, i, i, i, ctypes.POINTER(_Mask), dp]
+        lib.oracle_dropout_mask.restype = ctypes.c_int
         lib.oracle_set_threads.argtypes = [i]
         lib.oracle_get_threads.restype = i
         _lib = lib
@@ -110,9 +118,11 @@ class use_library:
         self.saved = _lib
         _load()  # make sure the argtypes template exists
         lib = ctypes.CDLL(self.so_path)
-        for name in ("oracle_fwd", "oracle_bwd", "oracle_probs"):
-            getattr(lib, name).argtypes = getattr(self.saved or _lib, name).argtypes
-            getattr(lib, name).restype = ctypes.c_int
+        for name in ("oracle_fwd", "oracle_bwd", "oracle_probs", "oracle_philox4x64",
+                     "oracle_dropout_mask"):
+            ref = getattr(self.saved or _lib, name)
+            getattr(lib, name).argtypes = ref.argtypes
+            getattr(lib, name).restype = ref.restype
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_get_threads.restype = ctypes.c_int
         _lib = lib
@@ -160,7 +170,7 @@ class _MaskHolder:
     """Keeps the numpy buffers a _Mask points to alive."""
 
     def __init__(self, B, N, Sq, Sk, causal, kv_len, mask, modality_ids,
-                 allow, allow_diag, bias=None):
+                 allow, allow_diag, bias=None, dropout=None):
         self.m = _Mask()
         self.m.causal = 1 if causal else 0
         self.keep = []
@@ -201,6 +211,14 @@ class _MaskHolder:
             self.keep.append(a4)
             self.m.add = a4.ctypes.data
             self.m.asb, self.m.ash, self.m.asq = N * Sq * Sk, Sq * Sk, Sk
+        if dropout is not None:
+            keep_prob, seed, offset = dropout
+            if not (0.0 < keep_prob <= 1.0):
+                raise ValueError("keep_prob must be in (0, 1]")
+            self.m.dropout = 1
+            self.m.keep_prob = float(keep_prob)
+            self.m.seed = int(seed) & ((1 << 64) - 1)
+            self.m.offset = int(offset) & ((1 << 64) - 1)
 
 
 def _prep(q, k, v, n_heads, layout):
@@ -216,19 +234,21 @@ def _prep(q, k, v, n_heads, layout):
 
 def fwd(q, k, v, scale, *, n_heads=None, layout="BNSD", causal=False,
         kv_len=None, mask=None, modality_ids=None, allow=((1, 1), (0, 1)),
-        allow_diag=False, slopes=None, bias=None):
+        allow_diag=False, slopes=None, bias=None, dropout=None):
     """Attention forward in fp64.  Returns (out, lse) as numpy arrays.
 
     ``out`` has the layout of ``q``; ``lse`` is [B, N, Sq] (natural log,
     -inf for rows with no allowed key).  ``mask`` is a bool/uint8 array
     broadcastable to [B, N, Sq, Sk] with 1 = may attend.  ``bias`` is a float
     array broadcastable to [B, N, Sq, Sk] added to the scores (a dense pse or
-    a float atten_mask; -inf entries mask their pair)."""
+    a float atten_mask; -inf entries mask their pair).  ``dropout`` is
+    ``(keep_prob, seed, offset)`` or None (the generator and mask layout are
+    in the header of oracle.c)."""
     if layout == "BSH" and n_heads is None:
         raise ValueError("BSH layout needs n_heads")
     q, k, v, B, N, Sq, Sk, D = _prep(q, k, v, n_heads, layout)
     mh = _MaskHolder(B, N, Sq, Sk, causal, kv_len, mask, modality_ids, allow,
-                     allow_diag, bias)
+                     allow_diag, bias, dropout)
     sl = None
     if slopes is not None:
         sl = np.ascontiguousarray(_f64(slopes).reshape(N))
@@ -245,14 +265,14 @@ def fwd(q, k, v, scale, *, n_heads=None, layout="BNSD", causal=False,
 
 def bwd(q, k, v, dout, scale, *, n_heads=None, layout="BNSD", causal=False,
         kv_len=None, mask=None, modality_ids=None, allow=((1, 1), (0, 1)),
-        allow_diag=False, slopes=None, bias=None):
+        allow_diag=False, slopes=None, bias=None, dropout=None):
     """Gradients (dq, dk, dv) of sum(dout * out) in fp64, layouts as the inputs."""
     if layout == "BSH" and n_heads is None:
         raise ValueError("BSH layout needs n_heads")
     q, k, v, B, N, Sq, Sk, D = _prep(q, k, v, n_heads, layout)
     do = _to_bnsd(_f64(dout), layout, n_heads)
     mh = _MaskHolder(B, N, Sq, Sk, causal, kv_len, mask, modality_ids, allow,
-                     allow_diag, bias)
+                     allow_diag, bias, dropout)
     sl = None
     if slopes is not None:
         sl = np.ascontiguousarray(_f64(slopes).reshape(N))
@@ -271,14 +291,14 @@ def bwd(q, k, v, dout, scale, *, n_heads=None, layout="BNSD", causal=False,
 
 def probs(q, k, scale, b, h, *, n_heads=None, layout="BNSD", causal=False,
           kv_len=None, mask=None, modality_ids=None, allow=((1, 1), (0, 1)),
-          allow_diag=False, slopes=None, bias=None):
+          allow_diag=False, slopes=None, bias=None, dropout=None):
     """Explicit probability matrix P [Sq, Sk] and lse [Sq] of one (b, h)."""
     q = _to_bnsd(_f64(q), layout, n_heads)
     k = _to_bnsd(_f64(k), layout, n_heads)
     B, N, Sq, D = q.shape
     Sk = k.shape[2]
     mh = _MaskHolder(B, N, Sq, Sk, causal, kv_len, mask, modality_ids, allow,
-                     allow_diag, bias)
+                     allow_diag, bias, dropout)
     sl = None
     if slopes is not None:
         sl = np.ascontiguousarray(_f64(slopes).reshape(N))
@@ -291,3 +311,23 @@ def probs(q, k, scale, b, h, *, n_heads=None, layout="BNSD", causal=False,
     if rc != 0:
         raise RuntimeError(f"oracle_probs failed ({rc})")
     return p, lse
+
+
+def philox4x64(counter, key):
+    """Philox-4x64-10 of one 4-word counter and 2-word key (uint64 words)."""
+    c = np.ascontiguousarray(np.asarray(counter, dtype=np.uint64).reshape(4))
+    k = np.ascontiguousarray(np.asarray(key, dtype=np.uint64).reshape(2))
+    out = np.zeros(4, dtype=np.uint64)
+    _load().oracle_philox4x64(c.ctypes.data, k.ctypes.data, out.ctypes.data)
+    return out
+
+
+def dropout_keep_mask(B, N, Sq, Sk, keep_prob, seed, offset):
+    """The dropout keep mask [B, N, Sq, Sk] (uint8, 1 = kept)."""
+    mh = _MaskHolder(B, N, Sq, Sk, False, None, None, None, ((1, 1), (1, 1)), False,
+                     None, (keep_prob, seed, offset))
+    keep = np.zeros((B, N, Sq, Sk), dtype=np.uint8)
+    rc = _load().oracle_dropout_mask(B, N, Sq, Sk, ctypes.byref(mh.m), keep.ctypes.data)
+    if rc != 0:
+        raise RuntimeError(f"oracle_dropout_mask failed ({rc})")
+    return keep

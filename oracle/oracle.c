@@ -31,6 +31,15 @@
  *                                       generalised to a 2x2 table)
  *   Disallowed scores are -inf (masked_fill with -inf, multimodal page,
  *   layer 2 flash_attention_with_mask).
+ *   Dropout (the guide's keep_prob, sec. 3.1/3.2; the unfused softmax ->
+ *   dropout -> matmul of sec. 1): p'_ij = p_ij * keep_ij / keep_prob with
+ *   keep_ij = [u_ij < round(keep_prob * 65536)], u_ij a 16-bit field of
+ *   Philox-4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers:
+ *   As Easy as 1, 2, 3", SC'11): counter (j / 16, i, b * N + h, 0), key
+ *   (seed, offset), field j mod 16 (word (j mod 16) / 4, bits 16 * (j mod 4)).
+ *   The pages fix only the retention probability; the generator, the
+ *   counter layout and the 16-bit threshold are this implementation's
+ *   reading.  O_i = sum_j p'_ij V_j; LSE is that of p (before dropout).
  *   m_i = max_allowed s_ij ; L_i = sum_allowed exp(s_ij - m_i)
  *   p_ij = exp(s_ij - m_i) / L_i  (0 where not allowed)
  *   O_i = sum_j p_ij V_j ; LSE_i = m_i + ln L_i
@@ -39,9 +48,10 @@
  *
  * Backward, from the same explicit P (the pages only say the gradient is
  * produced without storing the N x N matrix; the gradient itself is the
- * derivative of the forward definition above):
- *   dV_j = sum_i p_ij dO_i
- *   dP_ij = dO_i . V_j
+ * derivative of the forward definition above; f_ij = keep_ij / keep_prob
+ * with dropout, else 1):
+ *   dV_j = sum_i p_ij f_ij dO_i
+ *   dP_ij = f_ij (dO_i . V_j)
  *   Dl_i  = sum_j p_ij dP_ij
  *   dS_ij = p_ij (dP_ij - Dl_i)
  *   dQ_i  = scale * sum_j dS_ij K_j
@@ -70,7 +80,70 @@ typedef struct {
   const double* add;       /* dense additive term or NULL; element (b,h,i,j)
                               at b*asb + h*ash + i*asq + j */
   int64_t asb, ash, asq;
+  int dropout;             /* 1: apply dropout with keep_prob, seed, offset */
+  double keep_prob;
+  uint64_t seed, offset;
 } oracle_mask;
+
+/* Philox-4x64-10 (Salmon et al., SC'11): ten rounds of two 64x64->128
+ * multiplies by the round constants, the high halves xored with the other
+ * counter words and the key, the key bumped by the Weyl constants between
+ * rounds. */
+static void philox4x64_10(const uint64_t ctr[4], const uint64_t key[2], uint64_t out[4]) {
+  const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
+  const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
+  uint64_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+  uint64_t k0 = key[0], k1 = key[1];
+  for (int r = 0; r < 10; ++r) {
+    unsigned __int128 p0 = (unsigned __int128)M0 * x0;
+    unsigned __int128 p1 = (unsigned __int128)M1 * x2;
+    uint64_t hi0 = (uint64_t)(p0 >> 64), lo0 = (uint64_t)p0;
+    uint64_t hi1 = (uint64_t)(p1 >> 64), lo1 = (uint64_t)p1;
+    x0 = hi1 ^ x1 ^ k0;
+    x1 = lo1;
+    x2 = hi0 ^ x3 ^ k1;
+    x3 = lo0;
+    k0 += W0;
+    k1 += W1;
+  }
+  out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+void oracle_philox4x64(const uint64_t* ctr, const uint64_t* key, uint64_t* out) {
+  philox4x64_10(ctr, key, out);
+}
+
+/* keep_ij of the dropout definition in the header (1 = kept). */
+static int dropout_keep(const oracle_mask* m, int N, int b, int h, int i, int j) {
+  uint64_t ctr[4] = {(uint64_t)(j / 16), (uint64_t)i, (uint64_t)b * N + h, 0};
+  uint64_t key[2] = {m->seed, m->offset};
+  uint64_t w[4];
+  philox4x64_10(ctr, key, w);
+  int f = j % 16;
+  uint64_t u = (w[f / 4] >> (16 * (f % 4))) & 0xFFFFull;
+  double t = floor(m->keep_prob * 65536.0 + 0.5);
+  return (double)u < t;
+}
+
+/* f_ij = keep_ij / keep_prob with dropout, 1 without, for one (b, h). */
+static void dropout_factors(const oracle_mask* m, int N, int b, int h, int Sq, int Sk,
+                            double* f) {
+  for (int i = 0; i < Sq; ++i)
+    for (int j = 0; j < Sk; ++j)
+      f[(int64_t)i * Sk + j] =
+          (m && m->dropout) ? (dropout_keep(m, N, b, h, i, j) ? 1.0 / m->keep_prob : 0.0) : 1.0;
+}
+
+/* keep[b][h][i][j] (1 = kept) for tests. */
+int oracle_dropout_mask(int B, int N, int Sq, int Sk, const oracle_mask* m, uint8_t* keep) {
+  if (!m || !m->dropout) return 1;
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < N; ++h)
+      for (int i = 0; i < Sq; ++i)
+        for (int j = 0; j < Sk; ++j)
+          keep[(((int64_t)b * N + h) * Sq + i) * Sk + j] = (uint8_t)dropout_keep(m, N, b, h, i, j);
+  return 0;
+}
 
 static int oracle_threads = 0;
 
@@ -175,6 +248,10 @@ int oracle_fwd(int B, int N, int Sq, int Sk, int D, const double* q,
     }
     probs_one_head(b, h, Sq, Sk, D, qh, kh, slopes, m, scale, s, p,
                    lse + bh * Sq);
+    if (m && m->dropout) {   /* p' = p * f, kept in p (s is free now) */
+      dropout_factors(m, N, b, h, Sq, Sk, s);
+      for (int64_t e = 0; e < (int64_t)Sq * Sk; ++e) p[e] *= s[e];
+    }
     for (int i = 0; i < Sq; ++i)
       for (int d = 0; d < D; ++d) {
         double acc = 0.0;
@@ -217,21 +294,24 @@ int oracle_bwd(int B, int N, int Sq, int Sk, int D, const double* q,
       continue;
     }
     probs_one_head(b, h, Sq, Sk, D, qh, kh, slopes, m, scale, s, p, lse);
-    /* dV_j = sum_i p_ij dO_i */
+    double* f = s;   /* the dropout factors f_ij (1 without dropout) */
+    dropout_factors(m, N, b, h, Sq, Sk, f);
+    /* dV_j = sum_i p_ij f_ij dO_i */
     for (int j = 0; j < Sk; ++j)
       for (int d = 0; d < D; ++d) {
         double acc = 0.0;
         for (int i = 0; i < Sq; ++i)
-          acc += p[(int64_t)i * Sk + j] * doh[(int64_t)i * D + d];
+          acc += p[(int64_t)i * Sk + j] * f[(int64_t)i * Sk + j] * doh[(int64_t)i * D + d];
         dvh[(int64_t)j * D + d] = acc;
       }
-    /* dP_ij = dO_i . V_j ; Dl_i = sum_j p_ij dP_ij ; dS = p (dP - Dl) */
+    /* dP_ij = f_ij dO_i . V_j ; Dl_i = sum_j p_ij dP_ij ; dS = p (dP - Dl) */
     for (int i = 0; i < Sq; ++i) {
       double dl = 0.0;
       for (int j = 0; j < Sk; ++j) {
         double dp = 0.0;
         for (int d = 0; d < D; ++d)
           dp += doh[(int64_t)i * D + d] * vh[(int64_t)j * D + d];
+        dp *= f[(int64_t)i * Sk + j];
         ds[(int64_t)i * Sk + j] = dp; /* holds dP for now */
         dl += p[(int64_t)i * Sk + j] * dp;
       }

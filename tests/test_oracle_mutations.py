@@ -39,6 +39,12 @@ MUTATIONS = {
                       "if (m && m->add) val -= m->add[b * m->asb + h * m->ash + (int64_t)i * m->asq + j];"),
     "additive_neginf_kept": ("      if (val == -INFINITY) { /* an additive -inf masks the pair */",
                              "      if (0) { /* an additive -inf masks the pair */"),
+    "philox_round_order": ("    x0 = hi1 ^ x1 ^ k0;", "    x0 = hi0 ^ x1 ^ k0;"),
+    "dropout_counter_transposed": ("  uint64_t ctr[4] = {(uint64_t)(j / 16), (uint64_t)i, (uint64_t)b * N + h, 0};",
+                                   "  uint64_t ctr[4] = {(uint64_t)(i / 16), (uint64_t)j, (uint64_t)b * N + h, 0};"),
+    "dropout_no_rescale": ("(dropout_keep(m, N, b, h, i, j) ? 1.0 / m->keep_prob : 0.0)",
+                           "(dropout_keep(m, N, b, h, i, j) ? 1.0 : 0.0)"),
+    "dropout_dp_unmasked": ("        dp *= f[(int64_t)i * Sk + j];", "        dp *= 1.0;"),
     "dq_uses_q": ("acc += ds[(int64_t)i * Sk + j] * kh[(int64_t)j * D + d];",
                   "acc += ds[(int64_t)i * Sk + j] * qh[(int64_t)j * D + d];"),
 }
@@ -57,6 +63,9 @@ CHECKS = [
     lambda: pins.test_bias_of_zero_and_neginf_equals_the_bool_mask("bool"),
     lambda: pins.test_bias_constant_shift_moves_only_the_lse((2, 3, 6, 9)),
     pins.test_bias_q0_closed_form,
+    pins.test_philox_matches_numpy_bit_generator,
+    pins.test_dropout_mask_layout_matches_numpy_philox,
+    lambda: pins.test_dropout_matches_torch_autograd("causal"),
 ]
 
 

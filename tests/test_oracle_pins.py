@@ -536,3 +536,115 @@ def test_bias_bwd_finite_differences(mode):
             fd[idx] = (lp - lm) / (2 * h)
         err = np.abs(fd - g).max() / max(1.0, np.abs(g).max())
         assert err < 1e-6, (name, err)
+
+
+# ---------------------------------------------------------------- dropout (keep_prob < 1)
+# The guide's keep_prob (sec. 3.1/3.2).  The generator is Philox-4x64-10
+# (Salmon et al., SC'11), pinned to numpy's Philox bit generator (a library
+# implementation of the same published algorithm); the mask layout and the
+# dropout arithmetic are pinned to numpy and to torch autograd.
+
+def test_philox_matches_numpy_bit_generator():
+    rng = np.random.default_rng(160)
+    for _ in range(20):
+        ctr = rng.integers(1, 2**63, size=4, dtype=np.uint64)
+        key = rng.integers(0, 2**63, size=2, dtype=np.uint64) * np.uint64(2) + np.uint64(1)
+        prev = ctr.copy()
+        prev[0] -= np.uint64(1)          # numpy increments the counter before each block
+        want = np.random.Philox(counter=prev, key=key).random_raw(4)
+        np.testing.assert_array_equal(oracle.philox4x64(ctr, key), want)
+
+
+def test_dropout_mask_layout_matches_numpy_philox():
+    B, N, Sq, Sk = 2, 3, 5, 40
+    keep_prob, seed, offset = 0.6, 0x1234_5678_9ABC_DEF0, 77
+    keep = oracle.dropout_keep_mask(B, N, Sq, Sk, keep_prob, seed, offset)
+    t = math.floor(keep_prob * 65536 + 0.5)
+    for b in range(B):
+        for h in range(N):
+            for i in range(Sq):
+                for jg in range(0, Sk, 16):
+                    # counter (j / 16, i, b*N + h, 0) as a 256-bit integer;
+                    # numpy increments it before producing a block
+                    ctr = (jg // 16) | (i << 64) | ((b * N + h) << 128)
+                    words = np.random.Philox(counter=(ctr - 1) % (1 << 256), key=seed | (offset << 64)
+                                             ).random_raw(4)
+                    for j in range(jg, min(jg + 16, Sk)):
+                        f = j % 16
+                        u = (int(words[f // 4]) >> (16 * (f % 4))) & 0xFFFF
+                        assert keep[b, h, i, j] == (u < t), (b, h, i, j)
+
+
+def test_dropout_keep_rate_and_independence():
+    keep = oracle.dropout_keep_mask(2, 4, 128, 256, 0.85, 99, 3).astype(np.float64)
+    n = keep.size
+    assert abs(keep.mean() - 0.85) < 4 * math.sqrt(0.85 * 0.15 / n)
+    # neighbours along keys and along queries are uncorrelated
+    for a, b in ((keep[..., 1:], keep[..., :-1]), (keep[:, :, 1:], keep[:, :, :-1])):
+        c = np.corrcoef(a.ravel(), b.ravel())[0, 1]
+        assert abs(c) < 0.02
+    # another offset gives another mask
+    other = oracle.dropout_keep_mask(2, 4, 128, 256, 0.85, 99, 4)
+    assert np.mean(other != keep) > 0.2
+
+
+def test_keep_prob_one_reproduces_no_dropout():
+    B, N, Sq, Sk, D = 2, 2, 7, 9, 4
+    q, k, v, do = (_rand(s, 170 + n) for n, s in enumerate(
+        [(B, N, Sq, D), (B, N, Sk, D), (B, N, Sk, D), (B, N, Sq, D)]))
+    kw = dict(causal=False, kv_len=np.array([9, 5], dtype=np.int32), slopes=np.array([0.3, 0.1]))
+    o1, l1 = oracle.fwd(q, k, v, 0.5, **kw)
+    o2, l2 = oracle.fwd(q, k, v, 0.5, dropout=(1.0, 5, 6), **kw)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    for a, b in zip(oracle.bwd(q, k, v, do, 0.5, **kw),
+                    oracle.bwd(q, k, v, do, 0.5, dropout=(1.0, 5, 6), **kw)):
+        np.testing.assert_array_equal(a, b)
+
+
+@pytest.mark.parametrize("mode", ["none", "causal", "padding"])
+def test_dropout_matches_torch_autograd(mode):
+    B, N, Sq, Sk, D = 2, 2, 9, 21, 5
+    if mode == "causal":
+        Sk = Sq
+    keep_prob, seed, offset = 0.7, 2024, 11
+    gen = torch.Generator().manual_seed(180)
+    q, do = (torch.randn(B, N, Sq, D, dtype=torch.float64, generator=gen) for _ in range(2))
+    k, v = (torch.randn(B, N, Sk, D, dtype=torch.float64, generator=gen) for _ in range(2))
+    kw = _mask_kwargs(mode, B, N, Sq, Sk, seed=181)
+    allowed = _allowed_dense(mode, B, N, Sq, Sk, kw)
+    keep = torch.as_tensor(oracle.dropout_keep_mask(B, N, Sq, Sk, keep_prob, seed, offset)).bool()
+    qt, kt, vt = (t.clone().requires_grad_(True) for t in (q, k, v))
+    s = (qt @ kt.transpose(-1, -2)) * 0.45
+    p = torch.softmax(s.masked_fill(~allowed, float("-inf")), -1)
+    ref = (p * keep / keep_prob) @ vt
+    (ref * do).sum().backward()
+    out, lse = oracle.fwd(q, k, v, 0.45, dropout=(keep_prob, seed, offset), **kw)
+    np.testing.assert_allclose(out, ref.detach().numpy(), atol=1e-12, rtol=0)
+    ref_lse = torch.logsumexp(s.detach().masked_fill(~allowed, float("-inf")), -1).numpy()
+    np.testing.assert_allclose(lse, ref_lse, atol=1e-12, rtol=0)
+    dq, dk, dv = oracle.bwd(q, k, v, do, 0.45, dropout=(keep_prob, seed, offset), **kw)
+    np.testing.assert_allclose(dq, qt.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), atol=1e-12, rtol=0)
+
+
+def test_dropout_bwd_finite_differences():
+    B, N, S, D = 1, 2, 5, 3
+    q, k, v, do = (_rand((B, N, S, D), 190 + n) for n in range(4))
+    kw = dict(causal=True, slopes=np.array([0.4, 0.2]), dropout=(0.6, 7, 1))
+    dq, dk, dv = oracle.bwd(q, k, v, do, 0.8, **kw)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            args = {"q": q, "k": k, "v": v}
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args[name] = xp
+            lp = _loss(args["q"], args["k"], args["v"], do, 0.8, kw)
+            args[name] = xm
+            lm = _loss(args["q"], args["k"], args["v"], do, 0.8, kw)
+            fd[idx] = (lp - lm) / (2 * h)
+        err = np.abs(fd - g).max() / max(1.0, np.abs(g).max())
+        assert err < 1e-6, (name, err)
