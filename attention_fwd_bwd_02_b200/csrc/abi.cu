@@ -3,8 +3,9 @@
 //
 // The call follows npu_fusion_attention of the FlashAttentionScore guide
 // (sec. 3.1 call, sec. 3.2 parameter table): query/key/value, head count,
-// input layout BNSD or BSH, optional pse (ALiBi here), attention mask
-// (causal, key padding, bool, modality rule), scale and keep_prob (1.0 only).
+// input layout BNSD or BSH, optional pse (ALiBi slopes and / or a dense
+// additive term), attention mask (causal, key padding, bool, modality
+// rule), scale and keep_prob (dropout with the Philox mask of philox.cuh).
 #include <cuda_runtime.h>
 #include <math.h>
 #include <stdint.h>
@@ -48,12 +49,20 @@ fa_status check_shape(const fa_shape* s) {
 
 // Fills the kernel-side problem from the ABI arguments (after validation).
 fa_status make_problem(const fa_shape* s, const fa_pse* pse, const fa_mask* m,
-                       float scale, float keep_prob, Problem* p) {
+                       float scale, float keep_prob, const fa_dropout* drop, Problem* p) {
   fa_status st = check_shape(s);
   if (st != FA_OK) return st;
   if (!isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (!(keep_prob == 1.0f)) return FA_ERR_UNSUPPORTED;
+  if (!(keep_prob > 0.0f && keep_prob <= 1.0f)) return FA_ERR_INVALID_ARG;
   Problem q = {};
+  if (keep_prob < 1.0f) {
+    if (!drop) return FA_ERR_INVALID_ARG;
+    q.dropout = 1;
+    q.keep_t = uint32_t(floor(double(keep_prob) * 65536.0 + 0.5));
+    q.inv_keep = 1.0f / keep_prob;
+    q.seed = drop->seed;
+    q.offset = drop->offset;
+  }
   q.B = s->B;
   q.N = s->N;
   q.Sq = s->Sq;
@@ -196,10 +205,10 @@ namespace {
 // fa_fwd with test hooks (debug_flags, see the kernel's Problem).
 fa_status run_fwd(const fa_shape* shape, const void* q, const void* k,
                   const void* v, const fa_pse* pse, const fa_mask* mask,
-                  float scale, float keep_prob, void* out, float* lse,
-                  void* stream, uint32_t debug_flags) {
+                  float scale, float keep_prob, const fa_dropout* drop, void* out,
+                  float* lse, void* stream, uint32_t debug_flags) {
   Problem p;
-  fa_status st = make_problem(shape, pse, mask, scale, keep_prob, &p);
+  fa_status st = make_problem(shape, pse, mask, scale, keep_prob, drop, &p);
   if (st != FA_OK) return st;
   p.debug_flags = debug_flags;
   if (debug_flags && shape->dtype == FA_F32) return FA_ERR_UNSUPPORTED;
@@ -228,17 +237,18 @@ extern "C" {
 
 fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
                  const void* v, const fa_pse* pse, const fa_mask* mask,
-                 float scale, float keep_prob, void* out, float* lse,
-                 void* stream) {
-  return run_fwd(shape, q, k, v, pse, mask, scale, keep_prob, out, lse, stream, 0u);
+                 float scale, float keep_prob, const fa_dropout* dropout,
+                 void* out, float* lse, void* stream) {
+  return run_fwd(shape, q, k, v, pse, mask, scale, keep_prob, dropout, out, lse, stream, 0u);
 }
 
 fa_status fa_testing_fwd_withhold_q(const fa_shape* shape, const void* q,
                                     const void* k, const void* v,
                                     const fa_pse* pse, const fa_mask* mask,
-                                    float scale, float keep_prob, void* out,
+                                    float scale, float keep_prob,
+                                    const fa_dropout* dropout, void* out,
                                     float* lse, void* stream) {
-  return run_fwd(shape, q, k, v, pse, mask, scale, keep_prob, out, lse, stream,
+  return run_fwd(shape, q, k, v, pse, mask, scale, keep_prob, dropout, out, lse, stream,
                  fa::kDebugWithholdQ);
 }
 
@@ -252,10 +262,11 @@ size_t fa_bwd_workspace_size(const fa_shape* shape) {
 fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
                  const void* v, const void* out, const void* dout,
                  const float* lse, const fa_pse* pse, const fa_mask* mask,
-                 float scale, float keep_prob, void* dq, void* dk, void* dv,
-                 void* workspace, size_t workspace_bytes, void* stream) {
+                 float scale, float keep_prob, const fa_dropout* dropout,
+                 void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, void* stream) {
   Problem p;
-  fa_status st = make_problem(shape, pse, mask, scale, keep_prob, &p);
+  fa_status st = make_problem(shape, pse, mask, scale, keep_prob, dropout, &p);
   if (st != FA_OK) return st;
   if (p.B == 0 || p.N == 0) return FA_OK;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
@@ -314,7 +325,7 @@ size_t fa_mask_tile_map_size(const fa_shape* shape, const fa_mask* mask) {
 fa_status fa_build_mask_tile_map(const fa_shape* shape, const fa_mask* mask,
                                  uint8_t* tile_map, void* stream) {
   Problem p;
-  fa_status st = make_problem(shape, nullptr, mask, 1.0f, 1.0f, &p);
+  fa_status st = make_problem(shape, nullptr, mask, 1.0f, 1.0f, nullptr, &p);
   if (st != FA_OK) return st;
   if (!mask || !(mask->flags & FA_MASK_BOOL) || !tile_map) return FA_ERR_INVALID_ARG;
   cudaError_t e = fa::launch_tile_map(p, tile_map, static_cast<cudaStream_t>(stream));

@@ -33,6 +33,7 @@
 
 #include "fa_common.cuh"
 #include "launch.h"
+#include "philox.cuh"
 #include "ptx.cuh"
 #include "tma_host.h"
 
@@ -146,9 +147,9 @@ __device__ __forceinline__ int count_qtiles(const Problem& p, const KeyCtx& c) {
 __device__ __forceinline__ int col0_dq(int D, int wq) { return wq * (D / 4); }
 
 // kF16 selects fp16 operands (Q, K, V, dO, P, dS, dK, dV); bf16 otherwise.
-// kAdd: the problem has a dense additive term (p.add); a kernel of its own so
-// that the other kernels keep its registers.
-template <int D, bool kF16, bool kAdd>
+// kExt: the problem has a dense additive term (p.add) and / or dropout
+// (p.dropout); kernels of their own so that the others keep their registers.
+template <int D, bool kF16, bool kExt>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_sm100(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_k,
@@ -382,7 +383,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool has_alibi = p.slopes != nullptr;
     const bool causal = p.mask_flags & FA_MASK_CAUSAL;
     const bool fold = has_alibi && causal;  // ALiBi linear in i - j
-    constexpr bool has_add = kAdd;           // dense additive term (p.add)
+    const bool has_add = kExt && p.add != nullptr;  // dense additive term
+    const bool has_drop = kExt && p.dropout != 0;   // dropout mask
     const float abs_g = fold ? 0.f : -slope_l2;  // |i - j| form otherwise
     const int32_t* ids = (p.mask_flags & FA_MASK_MODALITY) ? p.ids + int64_t(c.b) * p.Sk : nullptr;
     const int id_j = (ids && j < p.Sk) ? (ids[j] & 1) : 0;
@@ -458,6 +460,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 32; ++e)
           av[e] = (a_in && q0 + e < p.Sq) ? __ldg(acol + int64_t(q0 + e) * p.a_sq) : 0.f;
       }
+      // Dropout keep bits of the 64 queries for key j (bit e: query q0 + e).
+      // Philox blocks hold 16 keys of one query, so each lane of a half-warp
+      // (16 consecutive keys) draws the blocks of 4 queries, and a ballot
+      // per key bit transposes them across the half-warp.
+      uint32_t kb[2] = {~0u, ~0u};
+      if (has_drop) {
+        const int hw = lane >> 4, rr = lane & 15;
+        const int jg = (c.k0 + wq * 32 + hw * 16) >> 4;
+        const int64_t bh = int64_t(c.b) * p.N + c.h;
+        kb[0] = kb[1] = 0u;
+#pragma unroll 1
+        for (int cq = 0; cq < 4; ++cq) {
+          const uint32_t m16 = dropout_bits16(p.seed, p.offset, p.keep_t, jg, q0 + 16 * cq + rr, bh);
+          uint32_t got = 0;
+#pragma unroll
+          for (int f = 0; f < 16; ++f) {
+            const uint32_t bal = __ballot_sync(~0u, (m16 >> f) & 1u);
+            if (f == rr) got = (bal >> (16 * hw)) & 0xFFFFu;
+          }
+          kb[cq >> 1] |= got << (16 * (cq & 1));
+        }
+      }
       const bool got_s = mbar_wait_s(BAR(C::bSFull + b), mine & 1, abort_addr);
       if (!__all_sync(~0u, got_s)) { ok = false; return false; }
       tc_fence_after();
@@ -513,7 +537,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < kBM; e += 2) {
           pf[e] = ex2_approx(__uint_as_float(sr[e >> 5][e & 31]));
           pf[e + 1] = ex2_approx(__uint_as_float(sr[e >> 5][(e & 31) + 1]));
-          pk[e >> 1] = pack_h2<kF16>(pf[e], pf[e + 1]);
+          if (has_drop)  // dV takes the kept, rescaled P
+            pk[e >> 1] = pack_h2<kF16>(((kb[e >> 5] >> (e & 31)) & 1u) ? pf[e] * p.inv_keep : 0.f,
+                                       ((kb[e >> 5] >> ((e & 31) + 1)) & 1u) ? pf[e + 1] * p.inv_keep : 0.f);
+          else
+            pk[e >> 1] = pack_h2<kF16>(pf[e], pf[e + 1]);
         }
         tmem_st32(tb + kColP, pk);
       }
@@ -528,8 +556,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int e = 0; e < 32; e += 2) {
           const int cc = hh * 32 + e;
           const float2 nd = ld_shared_f2(st + 4 * (kBM + cc));
-          const uint64_t t2 = fadd2(f2_pack(__uint_as_float(dr[e]), __uint_as_float(dr[e + 1])),
-                                    f2_pack(nd.x, nd.y));
+          float d0 = __uint_as_float(dr[e]), d1 = __uint_as_float(dr[e + 1]);
+          if (has_drop) {  // dP = mask / keep_prob * (dO V^T)
+            d0 = ((kb[hh] >> e) & 1u) ? d0 * p.inv_keep : 0.f;
+            d1 = ((kb[hh] >> (e + 1)) & 1u) ? d1 * p.inv_keep : 0.f;
+          }
+          const uint64_t t2 = fadd2(f2_pack(d0, d1), f2_pack(nd.x, nd.y));
           float s0, s1;
           f2_unpack(fmul2(t2, f2_pack(pf[cc], pf[cc + 1])), s0, s1);
           dsk[cc >> 1] = pack_h2<kF16>(s0, s1);
@@ -599,7 +631,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (tid == 0 && ld_shared_volatile(abort_addr)) atomicOr(p.status, 1u);
 }
 
-template <int D, bool kF16, bool kAdd>
+template <int D, bool kF16, bool kExt>
 cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
                          const void* v, const void* dout, const float* lse,
                          const float* delta, float* dq_acc, void* dk, void* dv,
@@ -620,12 +652,12 @@ cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
   // the increase waiting.
   static std::atomic<uint64_t> ready{0};
   e = once_per_device(ready, []() -> cudaError_t {
-    cudaError_t r = cudaFuncSetAttribute(bwd_sm100<D, kF16, kAdd>,
+    cudaError_t r = cudaFuncSetAttribute(bwd_sm100<D, kF16, kExt>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (r != cudaSuccess) return r;
     cudaFuncAttributes fa_attr;
-    if ((r = cudaFuncGetAttributes(&fa_attr, bwd_sm100<D, kF16, kAdd>)) != cudaSuccess) return r;
+    if ((r = cudaFuncGetAttributes(&fa_attr, bwd_sm100<D, kF16, kExt>)) != cudaSuccess) return r;
     return fa_attr.numRegs * kThreads <
                    2 * 128 * int(kRegsSoftmax) + 128 * int(kRegsDq) + 128 * int(kRegsControl)
                ? cudaErrorInvalidConfiguration
@@ -634,7 +666,7 @@ cudaError_t launch_bwd_d(const Problem& p, const void* q, const void* k,
   if (e != cudaSuccess) return e;
   dim3 grid((p.Sk + kBN - 1) / kBN, p.N, p.B);
   if (p.add && p.a_sb == 0) grid = dim3((p.Sk + kBN - 1) / kBN, p.B, p.N);
-  bwd_sm100<D, kF16, kAdd><<<grid, kThreads, C::kSmemBytes, st>>>(
+  bwd_sm100<D, kF16, kExt><<<grid, kThreads, C::kSmemBytes, st>>>(
       tq, tk, tv, tdo, tdq, p, lse, delta, static_cast<uint16_t*>(dk),
       static_cast<uint16_t*>(dv));
   return cudaGetLastError();
@@ -646,9 +678,9 @@ cudaError_t launch_bwd_sm100(const Problem& p, const void* q, const void* k,
                              const void* v, const void* dout, const float* lse,
                              const float* delta, float* dq_acc, void* dk, void* dv,
                              cudaStream_t st) {
-#define FA_BWD_CASE(HD, F16, ADD) \
-  if (p.D == HD && bool(p.f16) == F16 && (p.add != nullptr) == ADD) \
-    return launch_bwd_d<HD, F16, ADD>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
+#define FA_BWD_CASE(HD, F16, EXT) \
+  if (p.D == HD && bool(p.f16) == F16 && (p.add != nullptr || p.dropout != 0) == EXT) \
+    return launch_bwd_d<HD, F16, EXT>(p, q, k, v, dout, lse, delta, dq_acc, dk, dv, st);
   FA_BWD_CASE(64, false, false)
   FA_BWD_CASE(64, true, false)
   FA_BWD_CASE(128, false, false)

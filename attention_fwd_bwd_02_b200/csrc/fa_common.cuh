@@ -30,6 +30,10 @@ struct Problem {
   const float* add;         // dense additive term (pse tensor / float mask) or null
   int64_t a_sb, a_sh, a_sq; // its strides in elements (0 = broadcast)
   uint32_t add_vec;         // 1: 16-byte aligned rows, float4 loads allowed
+  uint32_t dropout;         // 1: keep_prob < 1 (mask from philox.cuh)
+  uint32_t keep_t;          // keep iff the 16-bit field < keep_t (0..65536)
+  float inv_keep;           // 1 / keep_prob
+  uint64_t seed, offset;    // Philox key
   uint32_t f16;             // tensor-core path: 1 = fp16 operands, 0 = bf16
   uint32_t debug_flags;     // test hooks, 0 in production (kDebug* below)
   unsigned int* status;     // device status word (bit 0: a wait timed out)

@@ -40,6 +40,7 @@
 #include "fa_common.cuh"
 #include "launch.h"
 #include "ptx.cuh"
+#include "philox.cuh"
 #include "sched.cuh"
 #include "tma_host.h"
 
@@ -298,9 +299,10 @@ __device__ __forceinline__ int tile_class(const Problem& p, const Item& c, int t
   return cls;
 }
 
-// kF16 selects fp16 operands (Q, K, V, P, out); bf16 otherwise.  kAdd: the
-// problem has a dense additive term (p.add), in a kernel of its own.
-template <int D, bool kF16, bool kAdd>
+// kF16 selects fp16 operands (Q, K, V, P, out); bf16 otherwise.  kExt: the
+// problem has a dense additive term (p.add) and / or dropout (p.dropout),
+// handled in kernels of their own so that the others keep their registers.
+template <int D, bool kF16, bool kExt>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_k,
@@ -597,7 +599,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tO = tmem + lane_base + C::kColO + t * D;
     const float sl2 = p.scale_log2;
     const bool has_alibi = p.slopes != nullptr;
-    constexpr bool has_add = kAdd;
+    const bool has_add = kExt && p.add != nullptr;
+    const bool has_drop = kExt && p.dropout != 0;
     int steps = 0, o_uses = 0;
     bool ok = true;
 
@@ -797,6 +800,14 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t pk[16];
+          // Dropout keep bits of these 32 keys (two Philox blocks of 16).
+          uint32_t kb32 = ~0u;
+          if (has_drop && row_real) {
+            const int jg = (k0 + 32 * q4) >> 4;
+            const int64_t bh = int64_t(c.b) * p.N + c.h;
+            kb32 = dropout_bits16(p.seed, p.offset, p.keep_t, jg, i, bh) |
+                   (dropout_bits16(p.seed, p.offset, p.keep_t, jg + 1, i, bh) << 16);
+          }
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const uint64_t s2 = f2_pack(__uint_as_float(sr[q4][e]), __uint_as_float(sr[q4][e + 1]));
@@ -810,6 +821,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               p1 = ex2_approx(a1);
             }
             rs2[(e >> 1) & 3] = fadd2(rs2[(e >> 1) & 3], f2_pack(p0, p1));
+            if (has_drop) {  // l sums P before dropout; P V takes the kept, rescaled P
+              p0 = ((kb32 >> e) & 1u) ? p0 * p.inv_keep : 0.f;
+              p1 = ((kb32 >> (e + 1)) & 1u) ? p1 * p.inv_keep : 0.f;
+            }
             pk[e >> 1] = pack_h2<kF16>(p0, p1);
           }
           tmem_st16(tS + q4 * 16, pk);
@@ -894,7 +909,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <int D, bool kF16, bool kAdd>
+template <int D, bool kF16, bool kExt>
 static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
                                 const void* v, void* out, float* lse,
                                 cudaStream_t st) {
@@ -909,12 +924,12 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   // with fewer registers per thread would leave the increase waiting.
   static std::atomic<uint64_t> ready{0};
   e = once_per_device(ready, []() -> cudaError_t {
-    cudaError_t r = cudaFuncSetAttribute(fwd_sm100<D, kF16, kAdd>,
+    cudaError_t r = cudaFuncSetAttribute(fwd_sm100<D, kF16, kExt>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (r != cudaSuccess) return r;
     cudaFuncAttributes fa_attr;
-    if ((r = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16, kAdd>)) != cudaSuccess) return r;
+    if ((r = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16, kExt>)) != cudaSuccess) return r;
     return fa_attr.numRegs < int(kRegsLaunch) ? cudaErrorInvalidConfiguration : cudaSuccess;
   });
   if (e != cudaSuccess) return e;
@@ -930,7 +945,7 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   group = group < 1 ? 1 : (group > p.B * p.N ? p.B * p.N : group);
   unsigned int* ctr = work_counter();
   if (!ctr) return cudaErrorUnknown;
-  fwd_sm100<D, kF16, kAdd><<<grid, kThreads, C::kSmemBytes, st>>>(
+  fwd_sm100<D, kF16, kExt><<<grid, kThreads, C::kSmemBytes, st>>>(
       tq, tk, tv, p, static_cast<uint16_t*>(out), lse, q_blocks, int(items), group, ctr);
   return cudaGetLastError();
 }
@@ -938,9 +953,9 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
 cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k,
                              const void* v, void* out, float* lse,
                              cudaStream_t st) {
-#define FA_FWD_CASE(HD, F16, ADD) \
-  if (p.D == HD && bool(p.f16) == F16 && (p.add != nullptr) == ADD) \
-    return launch_fwd_d<HD, F16, ADD>(p, q, k, v, out, lse, st);
+#define FA_FWD_CASE(HD, F16, EXT) \
+  if (p.D == HD && bool(p.f16) == F16 && (p.add != nullptr || p.dropout != 0) == EXT) \
+    return launch_fwd_d<HD, F16, EXT>(p, q, k, v, out, lse, st);
   FA_FWD_CASE(64, false, false)
   FA_FWD_CASE(64, true, false)
   FA_FWD_CASE(128, false, false)

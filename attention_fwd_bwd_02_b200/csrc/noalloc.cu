@@ -51,25 +51,25 @@ extern "C" fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q,
                                     const void* out, const void* dout,
                                     const float* lse, const fa_pse* pse,
                                     const fa_mask* mask, float scale,
-                                    float keep_prob, void* dq, void* dk,
-                                    void* dv, void* stream) {
+                                    float keep_prob, const fa_dropout* dropout,
+                                    void* dq, void* dk, void* dv, void* stream) {
   if (!shape) return FA_ERR_INVALID_ARG;
   if (shape->B == 0 || shape->N == 0 || shape->Sq == 0 || shape->Sk == 0) {
     // No (query, key) pair: fa_bwd needs no workspace for this shape, so
     // its result and status come without touching the scratch array.
     return fa_bwd(shape, q, k, v, out, dout, lse, pse, mask, scale, keep_prob,
-                  dq, dk, dv, nullptr, 0, stream);
+                  dropout, dq, dk, dv, nullptr, 0, stream);
   }
   const size_t need = fa_bwd_workspace_size(shape);
   if (need == 0 && shape->B > 0 && shape->N > 0 && shape->Sq > 0) {
     // An invalid shape: fa_bwd reports the precise status without touching
     // the device.
     return fa_bwd(shape, q, k, v, out, dout, lse, pse, mask, scale, keep_prob,
-                  dq, dk, dv, nullptr, 0, stream);
+                  dropout, dq, dk, dv, nullptr, 0, stream);
   }
   if (need > FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
   void* ws = nullptr;
   if (scratch_address(&ws) != cudaSuccess) return FA_ERR_CUDA;
   return fa_bwd(shape, q, k, v, out, dout, lse, pse, mask, scale, keep_prob,
-                dq, dk, dv, ws, FA_NOALLOC_SCRATCH_BYTES, stream);
+                dropout, dq, dk, dv, ws, FA_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -12,6 +12,7 @@
 #include <atomic>
 
 #include "fa_common.cuh"
+#include "philox.cuh"
 #include "launch.h"
 
 namespace fa {
@@ -96,6 +97,13 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
       const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
       const float alpha = expf(m[r] - m_use);  // 0 when m[r] = -inf
       const float pj = expf(s - m_use);        // 0 when masked
+      // P V takes the kept, rescaled p (philox.cuh); l sums p before dropout
+      const float pv = (p.dropout && j < p.Sk && pj != 0.f)
+                           ? (((dropout_bits16(p.seed, p.offset, p.keep_t, j >> 4, i,
+                                               int64_t(b) * p.N + h) >> (j & 15)) & 1u)
+                                  ? pj * p.inv_keep
+                                  : 0.f)
+                           : pj;
       float psum = pj;
 #pragma unroll
       for (int o = 16; o; o >>= 1) psum += __shfl_xor_sync(~0u, psum, o);
@@ -104,7 +112,7 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
 #pragma unroll
       for (int t = 0; t < kMaxD / 32; ++t) acc[r][t] *= alpha;
       for (int jj = 0; jj < kSimtKeys; ++jj) {
-        const float pb = __shfl_sync(~0u, pj, jj);
+        const float pb = __shfl_sync(~0u, pv, jj);
         if (pb == 0.f) continue;  // warp-uniform (broadcast value)
 #pragma unroll
         for (int t = 0; t < kMaxD / 32; ++t) {
@@ -203,7 +211,12 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         if (p.slopes) s += alibi_bias(p, h, i, j);
         if (p.add) s += add_term(p, b, h, i, j);
         pj = expf(s - lse_i);
-        dsj = pj * (dpd - dl_i);
+        float f = 1.f;  // dropout factor keep / keep_prob (philox.cuh)
+        if (p.dropout)
+          f = ((dropout_bits16(p.seed, p.offset, p.keep_t, j >> 4, i, int64_t(b) * p.N + h) >>
+                (j & 15)) & 1u) ? p.inv_keep : 0.f;
+        dsj = pj * (f * dpd - dl_i);
+        pj *= f;  // dV takes the kept, rescaled p
       }
       float dqv[kMaxD / 32];
 #pragma unroll

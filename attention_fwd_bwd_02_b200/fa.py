@@ -41,6 +41,10 @@ class FaError(RuntimeError):
         super().__init__(f"{what}: {name} ({status})" if what else f"{name} ({status})")
 
 
+class FaDropout(ctypes.Structure):
+    _fields_ = [("seed", ctypes.c_uint64), ("offset", ctypes.c_uint64)]
+
+
 class FaShape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("N", ctypes.c_int), ("Sq", ctypes.c_int),
                 ("Sk", ctypes.c_int), ("D", ctypes.c_int), ("layout", ctypes.c_int),
@@ -86,12 +90,13 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         vp, sz = ctypes.c_void_p, ctypes.c_size_t
         S, M, P = ctypes.POINTER(FaShape), ctypes.POINTER(FaMask), ctypes.POINTER(FaPse)
-        L.fa_fwd.argtypes = [S, vp, vp, vp, P, M, ctypes.c_float, ctypes.c_float,
+        R = ctypes.POINTER(FaDropout)
+        L.fa_fwd.argtypes = [S, vp, vp, vp, P, M, ctypes.c_float, ctypes.c_float, R,
                              vp, vp, vp]
         L.fa_bwd.argtypes = [S, vp, vp, vp, vp, vp, vp, P, M, ctypes.c_float,
-                             ctypes.c_float, vp, vp, vp, vp, sz, vp]
+                             ctypes.c_float, R, vp, vp, vp, vp, sz, vp]
         L.fa_bwd_noalloc.argtypes = [S, vp, vp, vp, vp, vp, vp, P, M, ctypes.c_float,
-                                     ctypes.c_float, vp, vp, vp, vp]
+                                     ctypes.c_float, R, vp, vp, vp, vp]
         L.fa_testing_fwd_withhold_q.argtypes = L.fa_fwd.argtypes
         L.fa_bwd_workspace_size.argtypes = [S]
         L.fa_bwd_workspace_size.restype = sz
@@ -252,6 +257,18 @@ def make_mask(shape: FaShape, *, causal=False, atten_mask=None, padding_kv_len=N
     return m if flags else None
 
 
+def make_dropout(keep_prob, seed, offset) -> Optional[FaDropout]:
+    """The Philox key of the dropout mask (include/fa.h, fa_dropout); None
+    when keep_prob == 1.  keep_prob < 1 needs an explicit seed."""
+    if not (0.0 < float(keep_prob) <= 1.0):
+        raise FaError(FA_ERR_INVALID_ARG, f"keep_prob {keep_prob} outside (0, 1]")
+    if float(keep_prob) == 1.0:
+        return None
+    if seed is None:
+        raise FaError(FA_ERR_INVALID_ARG, "keep_prob < 1 needs a dropout seed")
+    return FaDropout(int(seed) & (2**64 - 1), int(offset) & (2**64 - 1))
+
+
 def split_atten_mask(atten_mask):
     """(bool mask, additive term): a bool/uint8 atten_mask selects pairs
     (1 = may attend); a floating one is added to the scaled scores (the
@@ -310,7 +327,7 @@ def make_pse(pse: Optional[torch.Tensor], keep: _Keep, shape: Optional[FaShape] 
 def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
         padding_kv_len=None, atten_mask=None, scale=None, keep_prob=1.0, *,
         causal=False, modality_ids=None, allow=((1, 1), (0, 1)), allow_diag=False,
-        tile_map=None, out=None, lse=None,
+        tile_map=None, out=None, lse=None, seed=None, offset=0,
         _withhold_q=False) -> Tuple[torch.Tensor, torch.Tensor]:
     """Fused attention forward.  Returns (out, lse).
 
@@ -321,6 +338,8 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
     -inf; -inf masks the pair).  causal: the
     lower-triangular rule.  padding_kv_len: int [B] valid keys per batch.
     modality_ids [B, S] with the 2x2 ``allow`` table and ``allow_diag``.
+    keep_prob < 1: dropout with the Philox mask keyed by (seed, offset)
+    (include/fa.h, fa_dropout); pass the same values to bwd.
     scale has no default (pass 1/sqrt(D) explicitly)."""
     if scale is None:
         raise FaError(FA_ERR_INVALID_ARG, "scale must be given explicitly")
@@ -334,6 +353,7 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
                   padding_kv_len=padding_kv_len, modality_ids=modality_ids,
                   allow=allow, allow_diag=allow_diag, tile_map=tile_map, keep=keep)
     ps = make_pse(pse, keep, shape, add)
+    dr = make_dropout(keep_prob, seed, offset)
     if out is None:
         out = torch.empty_like(query)
     if lse is None:
@@ -346,7 +366,8 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
         st = entry(ctypes.byref(shape), _ptr(query), _ptr(key), _ptr(value),
                    None if ps is None else ctypes.byref(ps),
                    None if m is None else ctypes.byref(m),
-                   float(scale), float(keep_prob), _ptr(out), _ptr(lse),
+                   float(scale), float(keep_prob),
+                   None if dr is None else ctypes.byref(dr), _ptr(out), _ptr(lse),
                    _stream(query))
     _check(st, "fa_fwd")
     return out, lse
@@ -368,7 +389,7 @@ def bwd_workspace_size(shape: FaShape) -> int:
 def bwd(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
         pse=None, padding_kv_len=None, atten_mask=None, scale=None, keep_prob=1.0, *,
         causal=False, modality_ids=None, allow=((1, 1), (0, 1)), allow_diag=False,
-        tile_map=None, workspace=None, dq=None, dk=None, dv=None):
+        tile_map=None, workspace=None, dq=None, dk=None, dv=None, seed=None, offset=0):
     """Gradients (dq, dk, dv) of sum(dout * out), recomputing P from lse."""
     if scale is None:
         raise FaError(FA_ERR_INVALID_ARG, "scale must be given explicitly")
@@ -382,6 +403,7 @@ def bwd(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
                   padding_kv_len=padding_kv_len, modality_ids=modality_ids,
                   allow=allow, allow_diag=allow_diag, tile_map=tile_map, keep=keep)
     ps = make_pse(pse, keep, shape, add)
+    dr = make_dropout(keep_prob, seed, offset)
     need = bwd_workspace_size(shape)
     if workspace is None:
         workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=query.device)
@@ -399,7 +421,9 @@ def bwd(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
                           _ptr(out), _ptr(dout), _ptr(lse),
                           None if ps is None else ctypes.byref(ps),
                           None if m is None else ctypes.byref(m),
-                          float(scale), float(keep_prob), _ptr(dq), _ptr(dk), _ptr(dv),
+                          float(scale), float(keep_prob),
+                          None if dr is None else ctypes.byref(dr),
+                          _ptr(dq), _ptr(dk), _ptr(dv),
                           _ptr(workspace), ctypes.c_size_t(workspace.numel()),
                           _stream(query))
     _check(st, "fa_bwd")
@@ -412,7 +436,8 @@ NOALLOC_SCRATCH_BYTES = 32 << 20   # FA_NOALLOC_SCRATCH_BYTES of include/fa.h
 def bwd_noalloc(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
                 pse=None, padding_kv_len=None, atten_mask=None, scale=None, keep_prob=1.0,
                 *, causal=False, modality_ids=None, allow=((1, 1), (0, 1)),
-                allow_diag=False, tile_map=None, dq=None, dk=None, dv=None):
+                allow_diag=False, tile_map=None, dq=None, dk=None, dv=None, seed=None,
+                offset=0):
     """Backward through fa_bwd_noalloc: the library's fixed scratch array
     replaces the workspace, so the call allocates no scratch (the outputs
     dq, dk, dv are still the caller's).  Shapes whose workspace would exceed
@@ -429,6 +454,7 @@ def bwd_noalloc(query, key, value, out, dout, lse, head_num=None, input_layout="
                   padding_kv_len=padding_kv_len, modality_ids=modality_ids,
                   allow=allow, allow_diag=allow_diag, tile_map=tile_map, keep=keep)
     ps = make_pse(pse, keep, shape, add)
+    dr = make_dropout(keep_prob, seed, offset)
     dq = torch.empty_like(query) if dq is None else dq
     dk = torch.empty_like(key) if dk is None else dk
     dv = torch.empty_like(value) if dv is None else dv
@@ -440,7 +466,8 @@ def bwd_noalloc(query, key, value, out, dout, lse, head_num=None, input_layout="
                                   _ptr(out), _ptr(dout), _ptr(lse),
                                   None if ps is None else ctypes.byref(ps),
                                   None if m is None else ctypes.byref(m),
-                                  float(scale), float(keep_prob), _ptr(dq), _ptr(dk),
+                                  float(scale), float(keep_prob),
+                                  None if dr is None else ctypes.byref(dr), _ptr(dq), _ptr(dk),
                                   _ptr(dv), _stream(query))
     _check(st, "fa_bwd_noalloc")
     return dq, dk, dv

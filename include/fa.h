@@ -124,6 +124,21 @@ typedef struct {
   int64_t bias_stride_b, bias_stride_h, bias_stride_q;
 } fa_pse;
 
+/* Dropout (guide, sec. 3.1/3.2: keep_prob, "Dropout retention ratio",
+ * default 1.0 = no dropout).  With keep_prob < 1 each probability p_ij is
+ * kept with probability keep_prob and scaled by 1 / keep_prob, or zeroed;
+ * LSE stays that of the probabilities before dropout.  The keep mask is a
+ * function of (seed, offset, b, h, i, j) only, so the backward regenerates
+ * it exactly: element (b, h, i, j) is kept iff u < round(keep_prob * 65536)
+ * for u the 16-bit field j mod 16 (word (j mod 16) / 4, bits 16 * (j mod 4))
+ * of Philox-4x64-10 (Salmon et al., SC'11) at counter (j / 16, i, b*N + h, 0)
+ * and key (seed, offset).  Pass the same (seed, offset) to fa_bwd; advance
+ * `offset` (or change `seed`) between calls for fresh masks. */
+typedef struct {
+  uint64_t seed;
+  uint64_t offset;
+} fa_dropout;
+
 typedef struct {
   int B, N, Sq, Sk, D;          /* batch, heads (head_num), query and key
                                    lengths, head dim                         */
@@ -136,15 +151,17 @@ typedef struct {
  *   pse, mask : may be NULL (no bias / no mask).
  *   scale     : multiplies Q K^T (the 1/sqrt(d_k) of the guide's table; no
  *               default is assumed).
- *   keep_prob : must be 1.0 (no dropout); anything else returns
- *               FA_ERR_UNSUPPORTED.
+ *   keep_prob : retention probability in (0, 1]; 1 = no dropout.
+ *   dropout   : the mask's generator key (see fa_dropout); required when
+ *               keep_prob < 1, ignored (may be NULL) when keep_prob == 1.
  * Errors: FA_ERR_INVALID_ARG for null tensors, non-positive sizes, a
- * modality mask with Sq != Sk or a missing mask pointer; FA_ERR_UNSUPPORTED
- * for keep_prob != 1 or a bf16 / fp16 head dim other than 64 / 128. */
+ * modality mask with Sq != Sk, a missing mask pointer, keep_prob outside
+ * (0, 1] or a missing fa_dropout with keep_prob < 1; FA_ERR_UNSUPPORTED for
+ * a bf16 / fp16 head dim other than 64 / 128. */
 fa_status fa_fwd(const fa_shape* shape, const void* q, const void* k,
                  const void* v, const fa_pse* pse, const fa_mask* mask,
-                 float scale, float keep_prob, void* out, float* lse,
-                 void* stream);
+                 float scale, float keep_prob, const fa_dropout* dropout,
+                 void* out, float* lse, void* stream);
 
 /* Bytes of device workspace fa_bwd needs for this shape (fp32 dQ
  * accumulator plus per-row fp32 statistics).  0 on invalid shapes. */
@@ -154,12 +171,14 @@ size_t fa_bwd_workspace_size(const fa_shape* shape);
  * the forward's out and lse.  workspace must hold fa_bwd_workspace_size()
  * bytes (16-byte aligned); its contents on entry do not matter.  dq, dk, dv
  * are fully overwritten.  No gradient is produced for pse or the mask.
+ * keep_prob and dropout must be those of the forward that produced out.
  * Errors as fa_fwd, plus FA_ERR_INVALID_ARG for a short workspace. */
 fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
                  const void* v, const void* out, const void* dout,
                  const float* lse, const fa_pse* pse, const fa_mask* mask,
-                 float scale, float keep_prob, void* dq, void* dk, void* dv,
-                 void* workspace, size_t workspace_bytes, void* stream);
+                 float scale, float keep_prob, const fa_dropout* dropout,
+                 void* dq, void* dk, void* dv, void* workspace,
+                 size_t workspace_bytes, void* stream);
 
 /* Backward without a caller-provided workspace (no counterpart on the source
  * pages; an addition of this library).  Some callers cannot call cudaMalloc:
@@ -189,7 +208,8 @@ fa_status fa_bwd_noalloc(const fa_shape* shape, const void* q, const void* k,
                          const void* v, const void* out, const void* dout,
                          const float* lse, const fa_pse* pse,
                          const fa_mask* mask, float scale, float keep_prob,
-                         void* dq, void* dk, void* dv, void* stream);
+                         const fa_dropout* dropout, void* dq, void* dk,
+                         void* dv, void* stream);
 
 /* Bytes of the tile map for FA_MASK_BOOL with this shape and mask strides:
  * one byte per (b, h or 1 when mask_stride_h == 0, query tile, key tile). */

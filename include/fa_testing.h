@@ -25,7 +25,8 @@ extern "C" {
 fa_status fa_testing_fwd_withhold_q(const fa_shape* shape, const void* q,
                                     const void* k, const void* v,
                                     const fa_pse* pse, const fa_mask* mask,
-                                    float scale, float keep_prob, void* out,
+                                    float scale, float keep_prob,
+                                    const fa_dropout* dropout, void* out,
                                     float* lse, void* stream);
 
 #ifdef __cplusplus

@@ -31,7 +31,7 @@ def test_exports_every_declared_function(L):
 def test_testing_entry_validates_like_fwd(L):
     # Same validation as fa_fwd, before any device work; fp32 has no hook.
     args = lambda shape: (ctypes.byref(shape), FAKE, FAKE, FAKE, None, None,
-                          0.125, 1.0, FAKE, FAKE, None)
+                          0.125, 1.0, None, FAKE, FAKE, None)
     assert L.fa_testing_fwd_withhold_q(*args(_shape(D=96))) == fa.FA_ERR_UNSUPPORTED
     assert L.fa_testing_fwd_withhold_q(*args(_shape(B=-1))) == fa.FA_ERR_INVALID_ARG
     assert L.fa_testing_fwd_withhold_q(*args(_shape(dtype=fa.FA_F32))) == fa.FA_ERR_UNSUPPORTED
@@ -53,11 +53,12 @@ def _shape(**kw):
 FAKE = ctypes.c_void_p(0x10000)   # never dereferenced: validation fails first
 
 
-def _fwd(L, shape, pse=None, mask=None, scale=0.125, keep_prob=1.0, ptr=FAKE):
+def _fwd(L, shape, pse=None, mask=None, scale=0.125, keep_prob=1.0, ptr=FAKE, drop=None):
     return L.fa_fwd(ctypes.byref(shape), ptr, ptr, ptr,
                     None if pse is None else ctypes.byref(pse),
                     None if mask is None else ctypes.byref(mask),
-                    scale, keep_prob, ptr, ptr, None)
+                    scale, keep_prob, None if drop is None else ctypes.byref(drop),
+                    ptr, ptr, None)
 
 
 @pytest.mark.parametrize("kw,code", [
@@ -75,7 +76,11 @@ def test_shape_validation(L, kw, code):
 
 
 def test_keep_prob_and_scale(L):
-    assert _fwd(L, _shape(), keep_prob=0.9) == fa.FA_ERR_UNSUPPORTED
+    assert _fwd(L, _shape(), keep_prob=0.9) == fa.FA_ERR_INVALID_ARG   # no fa_dropout
+    for bad in (0.0, -0.5, 1.5, float("nan")):
+        assert _fwd(L, _shape(), keep_prob=bad, drop=fa.FaDropout(1, 2)) == fa.FA_ERR_INVALID_ARG
+    # a valid dropout set-up passes validation (an empty problem then returns FA_OK)
+    assert _fwd(L, _shape(B=0), keep_prob=0.9, drop=fa.FaDropout(1, 2)) == fa.FA_OK
     assert _fwd(L, _shape(), scale=float("nan")) == fa.FA_ERR_INVALID_ARG
     assert _fwd(L, _shape(), scale=float("inf")) == fa.FA_ERR_INVALID_ARG
 
@@ -125,17 +130,17 @@ def test_bwd_validation(L):
     assert ws >= rows * 128 * 4 + rows * 4
     assert L.fa_bwd_workspace_size(ctypes.byref(_shape(D=96))) == 0
     p = FAKE
-    rc = L.fa_bwd(ctypes.byref(s), p, p, p, p, p, p, None, None, 0.1, 0.5, p, p, p,
+    rc = L.fa_bwd(ctypes.byref(s), p, p, p, p, p, p, None, None, 0.1, 0.5, None, p, p, p,
                   p, ctypes.c_size_t(ws), None)
-    assert rc == fa.FA_ERR_UNSUPPORTED                  # keep_prob
-    rc = L.fa_bwd(ctypes.byref(s), p, p, p, p, p, p, None, None, 0.1, 1.0, p, p, p,
+    assert rc == fa.FA_ERR_INVALID_ARG                  # keep_prob < 1 without fa_dropout
+    rc = L.fa_bwd(ctypes.byref(s), p, p, p, p, p, p, None, None, 0.1, 1.0, None, p, p, p,
                   None, ctypes.c_size_t(ws), None)
     assert rc == fa.FA_ERR_INVALID_ARG                  # workspace missing
-    rc = L.fa_bwd(ctypes.byref(s), p, p, p, p, p, p, None, None, 0.1, 1.0, p, p, p,
+    rc = L.fa_bwd(ctypes.byref(s), p, p, p, p, p, p, None, None, 0.1, 1.0, None, p, p, p,
                   p, ctypes.c_size_t(ws - 16), None)
     assert rc == fa.FA_ERR_INVALID_ARG                  # workspace too small
     odd = ctypes.c_void_p(0x10008)
-    rc = L.fa_bwd(ctypes.byref(s), odd, p, p, p, p, p, None, None, 0.1, 1.0, p, p, p,
+    rc = L.fa_bwd(ctypes.byref(s), odd, p, p, p, p, p, None, None, 0.1, 1.0, None, p, p, p,
                   p, ctypes.c_size_t(ws), None)
     assert rc == fa.FA_ERR_INVALID_ARG                  # misaligned tensor
 
@@ -143,7 +148,7 @@ def test_bwd_validation(L):
 def test_misaligned_forward_pointer(L):
     odd = ctypes.c_void_p(0x10008)
     s = _shape()
-    rc = L.fa_fwd(ctypes.byref(s), odd, FAKE, FAKE, None, None, 0.1, 1.0, FAKE, FAKE, None)
+    rc = L.fa_fwd(ctypes.byref(s), odd, FAKE, FAKE, None, None, 0.1, 1.0, None, FAKE, FAKE, None)
     # Either the device lookup fails first on a machine without a GPU
     # (FA_ERR_CUDA) or the alignment check rejects it; never FA_OK.
     assert rc in (fa.FA_ERR_INVALID_ARG, fa.FA_ERR_CUDA)

@@ -56,7 +56,7 @@ def test_noalloc_matches_workspace_backward(D):
 def test_noalloc_empty_shape_is_a_no_op():
     s = fa.FaShape(0, 4, 128, 128, 64, fa.FA_LAYOUT_BNSD, fa.FA_BF16)
     assert fa.lib().fa_bwd_noalloc(s, None, None, None, None, None, None, None, None,
-                                   0.1, 1.0, None, None, None, None) == fa.FA_OK
+                                   0.1, 1.0, None, None, None, None, None) == fa.FA_OK
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
@@ -66,5 +66,5 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     p = torch.empty(16, dtype=torch.uint8, device="cuda")
     ptr = fa._ptr(p)
     rc = fa.lib().fa_bwd_noalloc(s, ptr, ptr, ptr, ptr, ptr, ptr, None, None, 0.1, 1.0,
-                                 ptr, ptr, ptr, None)
+                                 None, ptr, ptr, ptr, None)
     assert rc == fa.FA_ERR_UNSUPPORTED
