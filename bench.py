@@ -46,7 +46,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
 KERNEL_SOURCES = ["attention_fwd_bwd_02_b200/csrc/fwd_sm100.cu",
                   "attention_fwd_bwd_02_b200/csrc/bwd_sm100.cu",
                   "attention_fwd_bwd_02_b200/csrc/aux.cu",
-                  "attention_fwd_bwd_02_b200/csrc/ptx.cuh"]
+                  "attention_fwd_bwd_02_b200/csrc/ptx.cuh",
+                  "attention_fwd_bwd_02_b200/csrc/sched.cuh",
+                  "attention_fwd_bwd_02_b200/csrc/philox.cuh",
+                  "attention_fwd_bwd_02_b200/csrc/fa_common.cuh"]
 
 
 def peaks():
