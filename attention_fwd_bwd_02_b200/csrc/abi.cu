@@ -39,9 +39,10 @@ fa_status check_shape(const fa_shape* s) {
     return FA_ERR_INVALID_ARG;
   if (s->layout != FA_LAYOUT_BNSD && s->layout != FA_LAYOUT_BSH)
     return FA_ERR_INVALID_ARG;
-  if (s->dtype != FA_F32 && s->dtype != FA_BF16 && s->dtype != FA_F16)
+  if (s->dtype != FA_F32 && s->dtype != FA_BF16 && s->dtype != FA_F16 && s->dtype != FA_E4M3)
     return FA_ERR_INVALID_ARG;
   if (s->dtype != FA_F32 && s->D != 64 && s->D != 128) return FA_ERR_UNSUPPORTED;
+  if (s->dtype == FA_E4M3 && s->D != 128) return FA_ERR_UNSUPPORTED;
   if (s->dtype == FA_F32 && s->D > 128) return FA_ERR_UNSUPPORTED;
   if (s->B > 65535 || s->N > 65535) return FA_ERR_UNSUPPORTED;
   return FA_OK;
@@ -70,6 +71,7 @@ fa_status make_problem(const fa_shape* s, const fa_pse* pse, const fa_mask* m,
   q.D = s->D;
   q.layout = s->layout;
   q.f16 = s->dtype == FA_F16 ? 1u : 0u;
+  q.f8 = s->dtype == FA_E4M3 ? 1u : 0u;
   const int64_t H = int64_t(s->N) * s->D;
   if (s->layout == FA_LAYOUT_BNSD) {
     q.q_sb = int64_t(s->N) * s->Sq * s->D;
@@ -173,7 +175,8 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 size_t elem_size(const fa_shape* s) { return s->dtype == FA_F32 ? 4 : 2; }
 
-// Element type of the tensors for the helper kernels.
+// Element type of the tensors for the helper kernels (of the output for
+// e4m3 inputs, whose output is bf16).
 fa::Elem elem_of(const fa_shape* s) {
   return s->dtype == FA_F32 ? fa::Elem::kF32 : (s->dtype == FA_F16 ? fa::Elem::kF16 : fa::Elem::kBF16);
 }
@@ -268,6 +271,7 @@ fa_status fa_bwd(const fa_shape* shape, const void* q, const void* k,
   Problem p;
   fa_status st = make_problem(shape, pse, mask, scale, keep_prob, dropout, &p);
   if (st != FA_OK) return st;
+  if (shape->dtype == FA_E4M3) return FA_ERR_UNSUPPORTED;  // forward only
   if (p.B == 0 || p.N == 0) return FA_OK;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const size_t es = elem_size(shape);

@@ -35,6 +35,7 @@ struct Problem {
   float inv_keep;           // 1 / keep_prob
   uint64_t seed, offset;    // Philox key
   uint32_t f16;             // tensor-core path: 1 = fp16 operands, 0 = bf16
+  uint32_t f8;              // tensor-core forward: 1 = e4m3 operands (out bf16)
   uint32_t debug_flags;     // test hooks, 0 in production (kDebug* below)
   unsigned int* status;     // device status word (bit 0: a wait timed out)
 };

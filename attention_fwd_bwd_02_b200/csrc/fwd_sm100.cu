@@ -52,7 +52,7 @@ constexpr int kBM = 128;              // query rows per tile
 constexpr int kTiles = 2;             // query tiles per work item
 constexpr int kRows = kBM * kTiles;   // query rows per work item
 constexpr int kBN = 128;              // keys per tile
-constexpr int kBoxBytes = 128 * 128;  // one 128-row x 64-col 16-bit box
+constexpr int kBoxBytes = 128 * 128;  // one 128-row box of 128-byte rows (64 16-bit or 128 8-bit columns)
 constexpr int kThreads = 384;         // 3 warpgroups
 constexpr int kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;  // rescale O only if max grows > 2^8
@@ -103,12 +103,22 @@ __device__ __forceinline__ void exp2_fma_x2(float a0, float a1, float& p0, float
 // every exponential stays on the MUFU for now.
 constexpr uint32_t kSoftExpPairs = 0x0000u;
 
-template <int D>
+// Operand types of the tensor-core forward.
+constexpr int kOpBF16 = 0, kOpF16 = 1, kOpE4M3 = 2;
+
+template <int D, int kOp>
 struct FwdCfg {
-  static constexpr int kBoxes = D / 64;
+  // A 128-byte swizzle box holds 64 16-bit or 128 8-bit columns.
+  static constexpr int kBoxCols = kOp == kOpE4M3 ? 128 : 64;
+  static constexpr int kBoxes = D / kBoxCols;
   static constexpr int kTileBytes = kBoxes * kBoxBytes;  // 128 rows x D
-  static constexpr int kKStages = (D == 128) ? 2 : 3;
-  static constexpr int kVStages = (D == 128) ? 2 : 3;
+  static constexpr int kKStages = (kTileBytes > 16384) ? 2 : 3;
+  static constexpr int kVStages = (kTileBytes > 16384) ? 2 : 3;
+  // Q K^T and P V instructions per tile: K = 16 (16-bit) or 32 (e4m3)
+  // elements each, 32 bytes of a 128-byte swizzled row.
+  static constexpr int kQKSteps = kOp == kOpE4M3 ? D / 32 : D / 16;
+  static constexpr int kPVSteps = kOp == kOpE4M3 ? kBN / 32 : kBN / 16;
+  static constexpr int kPVRowBytes = (kOp == kOpE4M3 ? 32 : 16) * 128;  // V rows per P V step
   static constexpr int kColO = 256;  // O_t at kColO + t * D
   static constexpr int kSmemQ = 0;
   static constexpr int kSmemK = kTiles * kTileBytes;
@@ -299,17 +309,21 @@ __device__ __forceinline__ int tile_class(const Problem& p, const Item& c, int t
   return cls;
 }
 
-// kF16 selects fp16 operands (Q, K, V, P, out); bf16 otherwise.  kExt: the
-// problem has a dense additive term (p.add) and / or dropout (p.dropout),
-// handled in kernels of their own so that the others keep their registers.
-template <int D, bool kF16, bool kExt>
+// kOp: bf16, fp16 or e4m3 operands (Q, K, V and P; the output is bf16 for
+// e4m3, else the operand type; P is rounded to e4m3 before P V for e4m3).
+// kExt: the problem has a dense additive term (p.add) and / or dropout
+// (p.dropout), handled in kernels of their own so that the others keep
+// their registers.
+template <int D, int kOp, bool kExt>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100(const __grid_constant__ CUtensorMap tm_q,
               const __grid_constant__ CUtensorMap tm_k,
               const __grid_constant__ CUtensorMap tm_v, const Problem p,
               uint16_t* __restrict__ out, float* __restrict__ lse, int q_blocks,
               int n_items, int group, unsigned int* __restrict__ sched_ctr) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, kOp>;
+  constexpr bool kF16 = kOp == kOpF16;   // 16-bit type of P (16-bit ops) and of out
+  constexpr bool kF8 = kOp == kOpE4M3;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -413,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(BAR(C::bQFull + t), C::kTileBytes);
             for (int x = 0; x < C::kBoxes; ++x)
               tma_load_3d_s(sQa + t * C::kTileBytes + x * kBoxBytes, &tm_q, BAR(C::bQFull + t),
-                          col0 + 64 * x, c.q0[t], z);
+                          col0 + C::kBoxCols * x, c.q0[t], z);
           }
           ++q_uses[t];
         }
@@ -431,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(BAR(C::bKFull + sk), C::kTileBytes);
             for (int x = 0; x < C::kBoxes; ++x)
               tma_load_3d_s(sKa + sk * C::kTileBytes + x * kBoxBytes, &tm_k, BAR(C::bKFull + sk),
-                          col0 + 64 * x, kt * kBN, z);
+                          col0 + C::kBoxCols * x, kt * kBN, z);
           }
           ++kidx;
           if (lane == 0 && vidx >= C::kVStages)
@@ -441,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_arrive_expect_tx(BAR(C::bVFull + sv), C::kTileBytes);
             for (int x = 0; x < C::kBoxes; ++x)
               tma_load_3d_s(sVa + sv * C::kTileBytes + x * kBoxBytes, &tm_v, BAR(C::bVFull + sv),
-                          col0 + 64 * x, kt * kBN, z);
+                          col0 + C::kBoxCols * x, kt * kBN, z);
           }
           ++vidx;
         }
@@ -459,8 +473,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
     } else if (warp == 9) {
       // ---------------------------------------------------------- MMA
-      constexpr uint32_t idesc_qk = idesc_f32acc(128, kBN, 0, 0, kF16);
-      constexpr uint32_t idesc_pv = idesc_f32acc(128, D, 0, 1, kF16);
+      constexpr uint32_t idesc_qk =
+          kF8 ? idesc_f32acc_e4m3(128, kBN, 0, 0) : idesc_f32acc(128, kBN, 0, 0, kF16);
+      constexpr uint32_t idesc_pv =
+          kF8 ? idesc_f32acc_e4m3(128, D, 0, 1) : idesc_f32acc(128, D, 0, 1, kF16);
       // Operand descriptors as low halves (start address + leading offset);
       // every operand here has an 8-row stride of 1024 B (common high half).
       // Q and K are K-major (64-column boxes); V is N-major with a box of
@@ -492,9 +508,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t vd = v_lo + uint32_t(sv) * (C::kTileBytes >> 4);
         const uint32_t acc0 = item_pv[t] > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_ts_lh(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8, vd + kk * (2048 >> 4),
-                     kDescHi, idesc_pv, kk > 0 ? 1u : acc0);
+        for (int kk = 0; kk < C::kPVSteps; ++kk) {
+          // P columns 8 kk .. 8 kk + 7 hold keys 16 kk (16-bit) or 32 kk (e4m3) on
+          if (kF8)
+            umma_ts_lh_f8(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8,
+                          vd + kk * (C::kPVRowBytes >> 4), kDescHi, idesc_pv, kk > 0 ? 1u : acc0);
+          else
+            umma_ts_lh(tmem + C::kColO + t * D, tmem + t * 128 + kk * 8,
+                       vd + kk * (C::kPVRowBytes >> 4), kDescHi, idesc_pv, kk > 0 ? 1u : acc0);
+        }
         v_users -= 1u << (4 * sv);
         if (((v_users >> (4 * sv)) & 15u) == 0) umma_commit_s(BAR(C::bVEmpty + sv));
         pend_idx[t] = -1;
@@ -551,10 +573,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if ((t == 0 ? cls0 : cls1) == 0) continue;
                 const uint32_t qd = q_lo + t * (C::kTileBytes >> 4);
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
+                for (int kk = 0; kk < C::kQKSteps; ++kk) {
                   const uint32_t off = ((kk >> 2) * kBoxBytes + (kk & 3) * 32) >> 4;
-                  umma_ss_lh(tmem + t * 128, qd + off, kDescHi, kd + off, kDescHi, idesc_qk,
-                             kk > 0 ? 1u : 0u);
+                  if (kF8)
+                    umma_ss_lh_f8(tmem + t * 128, qd + off, kDescHi, kd + off, kDescHi, idesc_qk,
+                                  kk > 0 ? 1u : 0u);
+                  else
+                    umma_ss_lh(tmem + t * 128, qd + off, kDescHi, kd + off, kDescHi, idesc_qk,
+                               kk > 0 ? 1u : 0u);
                 }
                 umma_commit_s(BAR(C::bSFull + t));
                 pend_idx[t] = idx;
@@ -800,6 +826,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t pk[16];
+          uint32_t pk8[8];  // e4m3: keys 32 q4 .. 32 q4 + 31, four per column
           // Dropout keep bits of these 32 keys (two Philox blocks of 16).
           uint32_t kb32 = ~0u;
           if (has_drop && row_real) {
@@ -825,9 +852,17 @@ __global__ void __launch_bounds__(kThreads, 1)
               p0 = ((kb32 >> e) & 1u) ? p0 * p.inv_keep : 0.f;
               p1 = ((kb32 >> (e + 1)) & 1u) ? p1 * p.inv_keep : 0.f;
             }
-            pk[e >> 1] = pack_h2<kF16>(p0, p1);
+            if (kF8) {  // P <= 2^8 (the lazy rescale bound) fits e4m3 (max 448)
+              const uint32_t h = pack_e4m3x2(p0, p1);
+              pk8[e >> 2] = (e & 2) ? (pk8[e >> 2] | (h << 16)) : h;
+            } else {
+              pk[e >> 1] = pack_h2<kF16>(p0, p1);
+            }
           }
-          tmem_st16(tS + q4 * 16, pk);
+          if (kF8)
+            tmem_st8(tS + q4 * 8, pk8);
+          else
+            tmem_st16(tS + q4 * 16, pk);
         }
         if (item_steps > 0 && __any_sync(~0u, rescale)) {
           // S ready implies every earlier MMA (the previous P V) is complete,
@@ -909,7 +944,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <int D, bool kF16, bool kExt>
+template <int D, int kOp, bool kExt>
 static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
                                 const void* v, void* out, float* lse,
                                 cudaStream_t st) {
@@ -918,18 +953,18 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   if ((e = make_operand_map(&tq, q, p, p.Sq, 128)) != cudaSuccess) return e;
   if ((e = make_operand_map(&tk, k, p, p.Sk, 128)) != cudaSuccess) return e;
   if ((e = make_operand_map(&tv, v, p, p.Sk, 128)) != cudaSuccess) return e;
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, kOp>;
   // Shared-memory opt-in and the register check, once per device.  The
   // register split (setmaxnreg) draws on the launch allocation; a build
   // with fewer registers per thread would leave the increase waiting.
   static std::atomic<uint64_t> ready{0};
   e = once_per_device(ready, []() -> cudaError_t {
-    cudaError_t r = cudaFuncSetAttribute(fwd_sm100<D, kF16, kExt>,
+    cudaError_t r = cudaFuncSetAttribute(fwd_sm100<D, kOp, kExt>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::kSmemBytes);
     if (r != cudaSuccess) return r;
     cudaFuncAttributes fa_attr;
-    if ((r = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kF16, kExt>)) != cudaSuccess) return r;
+    if ((r = cudaFuncGetAttributes(&fa_attr, fwd_sm100<D, kOp, kExt>)) != cudaSuccess) return r;
     return fa_attr.numRegs < int(kRegsLaunch) ? cudaErrorInvalidConfiguration : cudaSuccess;
   });
   if (e != cudaSuccess) return e;
@@ -948,7 +983,7 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
   group = group < 1 ? 1 : (group > p.B * p.N ? p.B * p.N : group);
   unsigned int* ctr = work_counter();
   if (!ctr) return cudaErrorUnknown;
-  fwd_sm100<D, kF16, kExt><<<grid, kThreads, C::kSmemBytes, st>>>(
+  fwd_sm100<D, kOp, kExt><<<grid, kThreads, C::kSmemBytes, st>>>(
       tq, tk, tv, p, static_cast<uint16_t*>(out), lse, q_blocks, int(items), group, ctr);
   return cudaGetLastError();
 }
@@ -956,17 +991,20 @@ static cudaError_t launch_fwd_d(const Problem& p, const void* q, const void* k,
 cudaError_t launch_fwd_sm100(const Problem& p, const void* q, const void* k,
                              const void* v, void* out, float* lse,
                              cudaStream_t st) {
-#define FA_FWD_CASE(HD, F16, EXT) \
-  if (p.D == HD && bool(p.f16) == F16 && (p.add != nullptr || p.dropout != 0) == EXT) \
-    return launch_fwd_d<HD, F16, EXT>(p, q, k, v, out, lse, st);
-  FA_FWD_CASE(64, false, false)
-  FA_FWD_CASE(64, true, false)
-  FA_FWD_CASE(128, false, false)
-  FA_FWD_CASE(128, true, false)
-  FA_FWD_CASE(64, false, true)
-  FA_FWD_CASE(64, true, true)
-  FA_FWD_CASE(128, false, true)
-  FA_FWD_CASE(128, true, true)
+  const int op = p.f8 ? kOpE4M3 : (p.f16 ? kOpF16 : kOpBF16);
+#define FA_FWD_CASE(HD, OP, EXT) \
+  if (p.D == HD && op == OP && (p.add != nullptr || p.dropout != 0) == EXT) \
+    return launch_fwd_d<HD, OP, EXT>(p, q, k, v, out, lse, st);
+  FA_FWD_CASE(64, kOpBF16, false)
+  FA_FWD_CASE(64, kOpF16, false)
+  FA_FWD_CASE(128, kOpBF16, false)
+  FA_FWD_CASE(128, kOpF16, false)
+  FA_FWD_CASE(128, kOpE4M3, false)
+  FA_FWD_CASE(64, kOpBF16, true)
+  FA_FWD_CASE(64, kOpF16, true)
+  FA_FWD_CASE(128, kOpBF16, true)
+  FA_FWD_CASE(128, kOpF16, true)
+  FA_FWD_CASE(128, kOpE4M3, true)
 #undef FA_FWD_CASE
   return cudaErrorInvalidValue;
 }

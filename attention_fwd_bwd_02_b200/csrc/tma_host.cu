@@ -93,7 +93,7 @@ cudaError_t encode_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* b
 cudaError_t make_operand_map(CUtensorMap* map, const void* base,
                              const Problem& p, int S, int box_rows) {
   cuuint64_t dims[3], strides[2];
-  const cuuint64_t esz = 2;  // bf16 or fp16
+  const cuuint64_t esz = p.f8 ? 1 : 2;  // e4m3, or bf16 / fp16
   if (p.layout == FA_LAYOUT_BSH) {
     dims[0] = cuuint64_t(p.N) * p.D;
     dims[1] = cuuint64_t(S);
@@ -107,9 +107,12 @@ cudaError_t make_operand_map(CUtensorMap* map, const void* base,
     strides[0] = dims[0] * esz;
     strides[1] = dims[0] * dims[1] * esz;
   }
-  const cuuint32_t box[3] = {64u, cuuint32_t(box_rows), 1u};
-  return encode_3d(map, p.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                   base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  // 128-byte box rows: 64 16-bit or 128 8-bit columns
+  const cuuint32_t box[3] = {cuuint32_t(128 / esz), cuuint32_t(box_rows), 1u};
+  const CUtensorMapDataType dt = p.f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                      : (p.f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                               : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
+  return encode_3d(map, dt, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 cudaError_t make_f32_rows_map(CUtensorMap* map, const void* base, int cols,

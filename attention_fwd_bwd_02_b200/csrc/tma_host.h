@@ -9,9 +9,9 @@
 
 namespace fa {
 
-// Tensor map over a bf16 (p.f16 = 0) or fp16 (p.f16 = 1) operand with S
-// rows per head, read as boxes of
-// 64 columns x box_rows rows with 128-byte swizzle (the canonical K-major /
+// Tensor map over a bf16 (p.f16 = 0), fp16 (p.f16 = 1) or e4m3 (p.f8 = 1)
+// operand with S rows per head, read as boxes of 128-byte rows (64 16-bit or
+// 128 8-bit columns) x box_rows rows with 128-byte swizzle (the canonical K-major /
 // MN-major operand layout of tcgen05).  Coordinates (x, row, z):
 //   BNSD: x = column 0..D-1, z = b*N + h;   BSH: x = h*D + column, z = b.
 // Rows past S read as zeros.

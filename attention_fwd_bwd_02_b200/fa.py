@@ -28,7 +28,7 @@ TESTING_HEADER = os.path.join(os.path.dirname(_HERE), "include", "fa_testing.h")
 (FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT,
  FA_ERR_CONCURRENT) = range(6)
 FA_LAYOUT_BNSD, FA_LAYOUT_BSH = 0, 1
-FA_F32, FA_BF16, FA_F16 = 0, 1, 2
+FA_F32, FA_BF16, FA_F16, FA_E4M3 = 0, 1, 2, 3
 FA_MASK_CAUSAL, FA_MASK_KV_PADDING, FA_MASK_BOOL, FA_MASK_MODALITY = 1, 2, 4, 8
 FA_PSE_NONE, FA_PSE_ALIBI, FA_PSE_DENSE = 0, 1, 2
 FA_TILE_M = FA_TILE_N = 128
@@ -159,7 +159,14 @@ def _dtype_code(dt):
         return FA_F16
     if dt == torch.float32:
         return FA_F32
+    if dt == torch.float8_e4m3fn:
+        return FA_E4M3
     raise FaError(FA_ERR_UNSUPPORTED, f"dtype {dt}")
+
+
+def out_dtype(dt):
+    """dtype of the forward's output for operands of dtype dt (bf16 for e4m3)."""
+    return torch.bfloat16 if dt == torch.float8_e4m3fn else dt
 
 
 def make_shape(q, k, head_num, input_layout) -> FaShape:
@@ -340,6 +347,9 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
     modality_ids [B, S] with the 2x2 ``allow`` table and ``allow_diag``.
     keep_prob < 1: dropout with the Philox mask keyed by (seed, offset)
     (include/fa.h, fa_dropout); pass the same values to bwd.
+    float8_e4m3fn q/k/v (D = 128): the fp8 forward; out is bf16, and the
+    caller folds the dequantisation factors of q and k into scale and
+    multiplies out by that of v.
     scale has no default (pass 1/sqrt(D) explicitly)."""
     if scale is None:
         raise FaError(FA_ERR_INVALID_ARG, "scale must be given explicitly")
@@ -355,11 +365,13 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
     ps = make_pse(pse, keep, shape, add)
     dr = make_dropout(keep_prob, seed, offset)
     if out is None:
-        out = torch.empty_like(query)
+        out = torch.empty(query.shape, dtype=out_dtype(query.dtype), device=query.device)
     if lse is None:
         lse = torch.empty((shape.B, shape.N, shape.Sq), dtype=torch.float32,
                           device=query.device)
-    _check_operand(out, query.shape, "out", query)
+    _check_operand(out, query.shape, "out")
+    if out.dtype != out_dtype(query.dtype) or out.device != query.device:
+        raise FaError(FA_ERR_INVALID_ARG, f"out must be {out_dtype(query.dtype)} on q's device")
     _check_lse(lse, shape, query)
     entry = lib().fa_testing_fwd_withhold_q if _withhold_q else lib().fa_fwd
     with _on_device(query.device):
@@ -393,6 +405,8 @@ def bwd(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
     """Gradients (dq, dk, dv) of sum(dout * out), recomputing P from lse."""
     if scale is None:
         raise FaError(FA_ERR_INVALID_ARG, "scale must be given explicitly")
+    if query.dtype == torch.float8_e4m3fn:
+        raise FaError(FA_ERR_UNSUPPORTED, "the e4m3 path is forward only")
     shape = make_shape(query, key, head_num, input_layout)
     for t, n in ((query, "query"), (key, "key"), (value, "value"), (out, "out"),
                  (dout, "dout")):
@@ -444,6 +458,8 @@ def bwd_noalloc(query, key, value, out, dout, lse, head_num=None, input_layout="
     NOALLOC_SCRATCH_BYTES raise FA_ERR_UNSUPPORTED."""
     if scale is None:
         raise FaError(FA_ERR_INVALID_ARG, "scale must be given explicitly")
+    if query.dtype == torch.float8_e4m3fn:
+        raise FaError(FA_ERR_UNSUPPORTED, "the e4m3 path is forward only")
     shape = make_shape(query, key, head_num, input_layout)
     for t, n in ((query, "query"), (key, "key"), (value, "value"), (out, "out"),
                  (dout, "dout")):

@@ -114,15 +114,15 @@ def make_case(name, B, N, Sq, Sk, D, *, dtype=torch.bfloat16, layout="BNSD",
         n_text, n_image = modality
         assert n_text + n_image == Sq == Sk
         ids = modality_ids_text_image(B, n_text, n_image)
-    if dtype not in (torch.float32, torch.bfloat16, torch.float16):
+    if dtype not in (torch.float32, torch.bfloat16, torch.float16, torch.float8_e4m3fn):
         raise ValueError(f"unsupported dtype {dtype}")
 
     def cast(t):
         return t.to(dtype).contiguous()
 
     q, k, v = cast(q), cast(k), cast(v)
-    if dout is not None:
-        dout = cast(dout)
+    if dout is not None:  # e4m3 is forward only; its dO (unused) stays bf16
+        dout = dout.to(torch.bfloat16 if dtype == torch.float8_e4m3fn else dtype).contiguous()
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     return Case(name=name, B=B, N=N, Sq=Sq, Sk=Sk, D=D, dtype=dtype,

@@ -33,10 +33,16 @@
  *      FA_LAYOUT_BSH : q is [B][Sq][H], k and v are [B][Sk][H] with
  *                      H = N * D and head h at columns h*D .. h*D+D-1.
  *    All contiguous, D innermost.  out, dq, dk, dv use the layout and dtype
- *    of q, k, v.  lse is always fp32 [B][N][Sq].
+ *    of q, k, v (FA_E4M3: out is bf16).  lse is always fp32 [B][N][Sq].
  *  - Dtypes: FA_BF16 or FA_F16 (tensor-core path, D in {64, 128}), or FA_F32
  *    (fp32 FMA path, 1 <= D <= 128).  Accumulation is fp32 in all three; P
  *    and dS enter the tensor core in the operand type.
+ *  - FA_E4M3 (forward only, D = 128; the multimodal page's experimental
+ *    "pure fp8"): q, k, v are fp8 e4m3 (OCP E4M3, finite range +-448); the
+ *    tensor core computes S = Q K^T and O = P V in kind::f8f6f4 with fp32
+ *    accumulation, P rounded to e4m3 before P V.  Per-tensor dequantisation
+ *    factors are the caller's: fold those of q and k into `scale`, and
+ *    multiply the bf16 out by that of v.  fa_bwd returns FA_ERR_UNSUPPORTED.
  *  - Tensor pointers must be 16-byte aligned.
  */
 #ifndef FA_B200_H
@@ -61,7 +67,7 @@ typedef enum {
 } fa_status;
 
 typedef enum { FA_LAYOUT_BNSD = 0, FA_LAYOUT_BSH = 1 } fa_layout;
-typedef enum { FA_F32 = 0, FA_BF16 = 1, FA_F16 = 2 } fa_dtype;
+typedef enum { FA_F32 = 0, FA_BF16 = 1, FA_F16 = 2, FA_E4M3 = 3 } fa_dtype;
 
 /* Mask rules (bit flags, combinable).  A key j is visible to query i when
  * every active rule allows it.  Disallowed scores are -inf before the

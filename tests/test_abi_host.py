@@ -70,6 +70,8 @@ def _fwd(L, shape, pse=None, mask=None, scale=0.125, keep_prob=1.0, ptr=FAKE, dr
     (dict(layout=7), fa.FA_ERR_INVALID_ARG),
     (dict(dtype=5), fa.FA_ERR_INVALID_ARG),
     (dict(N=70000), fa.FA_ERR_UNSUPPORTED),
+    (dict(D=64, dtype=fa.FA_E4M3), fa.FA_ERR_UNSUPPORTED),  # e4m3 is D = 128 only
+    (dict(dtype=4), fa.FA_ERR_INVALID_ARG),
 ])
 def test_shape_validation(L, kw, code):
     assert _fwd(L, _shape(**kw)) == code
@@ -143,6 +145,14 @@ def test_bwd_validation(L):
     rc = L.fa_bwd(ctypes.byref(s), odd, p, p, p, p, p, None, None, 0.1, 1.0, None, p, p, p,
                   p, ctypes.c_size_t(ws), None)
     assert rc == fa.FA_ERR_INVALID_ARG                  # misaligned tensor
+
+
+def test_e4m3_backward_is_unsupported(L):
+    s = _shape(dtype=fa.FA_E4M3)
+    p = FAKE
+    rc = L.fa_bwd(ctypes.byref(s), p, p, p, p, p, p, None, None, 0.1, 1.0, None, p, p, p,
+                  p, ctypes.c_size_t(1 << 30), None)
+    assert rc == fa.FA_ERR_UNSUPPORTED
 
 
 def test_misaligned_forward_pointer(L):
