@@ -212,6 +212,17 @@ def _check_lse(lse, shape, like):
                       f"lse must be a contiguous fp32 [B, N, Sq] tensor on q's device")
 
 
+def check_side_inputs(device, **tensors):
+    """Every tensor the kernels read through a pointer (masks, lengths, ids,
+    tile map, slopes, dense term) must live on the operands' device: a host
+    or another GPU's pointer would be read by the kernel itself."""
+    for name, t in tensors.items():
+        if t is None:
+            continue
+        if not t.is_cuda or t.device != torch.device(device):
+            raise FaError(FA_ERR_INVALID_ARG, f"{name} must be a CUDA tensor on {device}")
+
+
 class _Keep:
     """Holds tensors that a ctypes struct points to."""
 
@@ -358,6 +369,8 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
     _check_operand(key, None, "key", query)
     _check_operand(value, key.shape, "value", query)
     keep = _Keep()
+    check_side_inputs(query.device, pse=pse, atten_mask=atten_mask, padding_kv_len=padding_kv_len,
+                      modality_ids=modality_ids, tile_map=tile_map)
     atten_mask, add = split_atten_mask(atten_mask)
     m = make_mask(shape, causal=causal, atten_mask=atten_mask,
                   padding_kv_len=padding_kv_len, modality_ids=modality_ids,
@@ -412,6 +425,8 @@ def bwd(query, key, value, out, dout, lse, head_num=None, input_layout="BNSD",
                  (dout, "dout")):
         _check_operand(t, None, n, query)
     keep = _Keep()
+    check_side_inputs(query.device, pse=pse, atten_mask=atten_mask, padding_kv_len=padding_kv_len,
+                      modality_ids=modality_ids, tile_map=tile_map)
     atten_mask, add = split_atten_mask(atten_mask)
     m = make_mask(shape, causal=causal, atten_mask=atten_mask,
                   padding_kv_len=padding_kv_len, modality_ids=modality_ids,
@@ -465,6 +480,8 @@ def bwd_noalloc(query, key, value, out, dout, lse, head_num=None, input_layout="
                  (dout, "dout")):
         _check_operand(t, None, n, query)
     keep = _Keep()
+    check_side_inputs(query.device, pse=pse, atten_mask=atten_mask, padding_kv_len=padding_kv_len,
+                      modality_ids=modality_ids, tile_map=tile_map)
     atten_mask, add = split_atten_mask(atten_mask)
     m = make_mask(shape, causal=causal, atten_mask=atten_mask,
                   padding_kv_len=padding_kv_len, modality_ids=modality_ids,
@@ -492,6 +509,7 @@ def bwd_noalloc(query, key, value, out, dout, lse, head_num=None, input_layout="
 def build_tile_map(atten_mask, query, key, head_num=None, input_layout="BNSD"):
     """Tile classification of a bool mask (one byte per 128 x 128 tile)."""
     shape = make_shape(query, key, head_num, input_layout)
+    check_side_inputs(query.device, query=query, atten_mask=atten_mask)
     keep = _Keep()
     m = make_mask(shape, atten_mask=atten_mask, keep=keep)
     n = int(lib().fa_mask_tile_map_size(ctypes.byref(shape), ctypes.byref(m)))
@@ -505,6 +523,7 @@ def build_tile_map(atten_mask, query, key, head_num=None, input_layout="BNSD"):
 
 def build_modality_mask(modality_ids, allow=((1, 1), (0, 1)), allow_diag=False):
     """Explicit cross-modal bool mask [B, S, S] (uint8, 1 = may attend)."""
+    check_side_inputs(modality_ids.device, modality_ids=modality_ids)
     ids = modality_ids.to(torch.int32).contiguous()
     B, S = ids.shape
     mask = torch.empty((B, S, S), dtype=torch.uint8, device=ids.device)
