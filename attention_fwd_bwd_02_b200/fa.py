@@ -309,10 +309,10 @@ def _dense_term(t: torch.Tensor, shape: FaShape, keep: _Keep):
         raise FaError(FA_ERR_INVALID_ARG,
                       f"dense pse / float mask of shape {tuple(t.shape)} does not broadcast "
                       f"to [{shape.B}, {shape.N}, {shape.Sq}, {shape.Sk}]")
-    if a.stride(-1) != 1 or a.stride(-2) < shape.Sk or \
-            (a.shape[0] > 1 and a.stride(0) <= 0) or (a.shape[1] > 1 and a.stride(1) <= 0):
+    if a.stride(-1) != 1 or a.stride(-2) < shape.Sk:
         a = a.contiguous()
     keep.items.append(a)
+    # a size-1 or expanded (stride 0) batch / head dimension is a broadcast
     sb = 0 if a.shape[0] == 1 else a.stride(0)
     sh = 0 if a.shape[1] == 1 else a.stride(1)
     return a.data_ptr(), sb, sh, a.stride(2)
