@@ -132,3 +132,17 @@ def test_both_dense_terms_are_rejected():
     t = torch.zeros(1, 1, 64, 64, device="cuda")
     with pytest.raises(fa.FaError):
         fa.fwd(dev["q"], dev["k"], dev["v"], 1, "BNSD", scale=c.scale, pse=t, atten_mask=t)
+
+
+def test_expanded_term_equals_its_copy():
+    """An expanded (stride-0) batch dimension is passed as a broadcast: the
+    result equals that of the materialised copy bit for bit."""
+    c = I.make_case("dense_expand", 3, 2, 130, 200, 64, seed=157)
+    dev = P.to_dev(c)
+    base = _term((1, 2, 130, 200), 158).cuda()
+    expanded = base.expand(3, 2, 130, 200)
+    assert expanded.stride(0) == 0
+    o1, l1 = fa.fwd(dev["q"], dev["k"], dev["v"], c.N, scale=c.scale, pse=expanded)
+    o2, l2 = fa.fwd(dev["q"], dev["k"], dev["v"], c.N, scale=c.scale, pse=expanded.contiguous())
+    fa.sync_status()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
