@@ -623,6 +623,68 @@ def run_configs(args):
         del dev, out, lse, ws
 
 
+def run_variant(args):
+    """Times one NEXT-row variant of the headline workload (causal B=4 N=32
+    S=2048 D=128) and prints one JSON line (not the main line):
+      e4m3    -- the fp8 forward (fa_fwd with e4m3 q, k, v; bf16 out);
+      dense   -- fa_fwd + fa_bwd with a dense [1, N, S, S] fp32 term;
+      dropout -- fa_fwd + fa_bwd with keep_prob = 0.9."""
+    import torch
+    from attention_fwd_bwd_02_b200 import fa
+    from attention_fwd_bwd_02_b200 import inputs as I
+    pk, pk_kind = peaks()
+    peak = pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    case = I.config2()
+    dev = torch.device("cuda")
+    q, k, v, do = (t.to(dev) for t in (case.q, case.k, case.v, case.dout))
+    kw = dict(scale=case.scale, causal=True)
+    with_bwd = args.variant != "e4m3"
+    if args.variant == "e4m3":
+        q, k, v = (t.to(torch.float8_e4m3fn) for t in (q, k, v))
+        peak = 2.0 * peak   # e4m3 dense rate is twice bf16's (4.5 vs 2.25 PFLOP/s nominal)
+    elif args.variant == "dense":
+        g = torch.Generator(device=dev).manual_seed(3)
+        kw["pse"] = torch.randn(1, N, S, S, device=dev, generator=g)
+    else:
+        kw.update(keep_prob=0.9, seed=1234, offset=0)
+    out, lse = fa.fwd(q, k, v, N, **kw)
+    ws = torch.empty(fa.bwd_workspace_size(fa.make_shape(q, k, N, "BNSD")), dtype=torch.uint8,
+                     device=dev)
+    step = [lambda: fa.fwd(q, k, v, N, out=out, lse=lse, **kw)]
+    if with_bwd:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        step.append(lambda: fa.bwd(q, k, v, out, do, lse, N, workspace=ws, dq=dq, dk=dk,
+                                   dv=dv, **kw))
+    for _ in range(args.warmup):
+        for f in step:
+            f()
+    fa.sync_status(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for s_ in range(args.steps):
+        ev[s_][0].record()
+        step[0]()
+        ev[s_][1].record()
+        if with_bwd:
+            step[1]()
+        ev[s_][2].record()
+    torch.cuda.synchronize()
+    fa.sync_status(dev)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps
+    line = {"variant": args.variant, "metric": METRIC, "unit": "TFLOP/s",
+            "config": {"workload": WORKLOAD, "B": B, "N": N, "S": S, "D": D},
+            "steps": args.steps, "warmup": args.warmup,
+            "fwd_ms": round(fwd_ms, 4), "fwd_tflops": round(FWD_FLOPS / (fwd_ms * 1e-3) / 1e12, 2),
+            "fwd_frac_of_peak": round(FWD_FLOPS / (fwd_ms * 1e-3) / 1e12 / peak, 4),
+            "peak": peak, "peak_kind": f"{pk_kind} bf16_tflops (burst)"
+                                       + (" x 2 for e4m3" if args.variant == "e4m3" else "")}
+    if with_bwd:
+        bwd_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps
+        line.update(bwd_ms=round(bwd_ms, 4),
+                    bwd_tflops=round(BWD_FLOPS / (bwd_ms * 1e-3) / 1e12, 2))
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -638,6 +700,9 @@ def main():
     ap.add_argument("--configs", action="store_true",
                     help="instead of the main line, time every workload of the "
                          "source pages (one JSON line each)")
+    ap.add_argument("--variant", choices=["e4m3", "dense", "dropout"],
+                    help="instead of the main line, time one variant of the "
+                         "headline workload (fp8 forward, dense term, dropout)")
     args = ap.parse_args()
     if args.impl == "ours":
         args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
@@ -645,6 +710,8 @@ def main():
         run_reference(args)
     elif args.configs:
         run_configs(args)
+    elif args.variant:
+        run_variant(args)
     else:
         run_ours(args)
 
