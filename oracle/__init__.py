@@ -94,8 +94,8 @@ def _load():
         lib.oracle_probs.argtypes = [i, i, i, i, i, i, i, dp, dp, dp,
                                      ctypes.POINTER(_Mask), ctypes.c_double, dp, dp]
         lib.oracle_probs.restype = ctypes.c_int
-        lib.oracle_philox4x64.argtypes = [dp, dp, dp]
-        lib.oracle_philox4x64.restype = None
+        lib.oracle_philox4x32.argtypes = [dp, dp, dp]
+        lib.oracle_philox4x32.restype = None
         lib.oracle_dropout_mask.argtypes = [i, i, i, i, ctypes.POINTER(_Mask), dp]
         lib.oracle_dropout_mask.restype = ctypes.c_int
         lib.oracle_set_threads.argtypes = [i]
@@ -118,7 +118,7 @@ class use_library:
         self.saved = _lib
         _load()  # make sure the argtypes template exists
         lib = ctypes.CDLL(self.so_path)
-        for name in ("oracle_fwd", "oracle_bwd", "oracle_probs", "oracle_philox4x64",
+        for name in ("oracle_fwd", "oracle_bwd", "oracle_probs", "oracle_philox4x32",
                      "oracle_dropout_mask"):
             ref = getattr(self.saved or _lib, name)
             getattr(lib, name).argtypes = ref.argtypes
@@ -313,12 +313,12 @@ def probs(q, k, scale, b, h, *, n_heads=None, layout="BNSD", causal=False,
     return p, lse
 
 
-def philox4x64(counter, key):
-    """Philox-4x64-10 of one 4-word counter and 2-word key (uint64 words)."""
-    c = np.ascontiguousarray(np.asarray(counter, dtype=np.uint64).reshape(4))
-    k = np.ascontiguousarray(np.asarray(key, dtype=np.uint64).reshape(2))
-    out = np.zeros(4, dtype=np.uint64)
-    _load().oracle_philox4x64(c.ctypes.data, k.ctypes.data, out.ctypes.data)
+def philox4x32(counter, key):
+    """Philox-4x32-10 of one 4-word counter and 2-word key (uint32 words)."""
+    c = np.ascontiguousarray(np.asarray(counter, dtype=np.uint32).reshape(4))
+    k = np.ascontiguousarray(np.asarray(key, dtype=np.uint32).reshape(2))
+    out = np.zeros(4, dtype=np.uint32)
+    _load().oracle_philox4x32(c.ctypes.data, k.ctypes.data, out.ctypes.data)
     return out
 
 

@@ -34,9 +34,11 @@
  *   Dropout (the guide's keep_prob, sec. 3.1/3.2; the unfused softmax ->
  *   dropout -> matmul of sec. 1): p'_ij = p_ij * keep_ij / keep_prob with
  *   keep_ij = [u_ij < round(keep_prob * 65536)], u_ij a 16-bit field of
- *   Philox-4x64-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers:
- *   As Easy as 1, 2, 3", SC'11): counter (j / 16, i, b * N + h, 0), key
- *   (seed, offset), field j mod 16 (word (j mod 16) / 4, bits 16 * (j mod 4)).
+ *   Philox-4x32-10 (Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers:
+ *   As Easy as 1, 2, 3", SC'11) with key (seed mod 2^32, seed / 2^32) and
+ *   counter words (c0, c1) = offset + j / 8 (a 64-bit block index, mod 2^64),
+ *   c2 = i, c3 = (b * N + h) mod 2^32; field j mod 8 is word (j mod 8) / 2,
+ *   bits 16 * (j mod 2).
  *   The pages fix only the retention probability; the generator, the
  *   counter layout and the 16-bit threshold are this implementation's
  *   reading.  O_i = sum_j p'_ij V_j; LSE is that of p (before dropout).
@@ -85,20 +87,20 @@ typedef struct {
   uint64_t seed, offset;
 } oracle_mask;
 
-/* Philox-4x64-10 (Salmon et al., SC'11): ten rounds of two 64x64->128
- * multiplies by the round constants, the high halves xored with the other
+/* Philox-4x32-10 (Salmon et al., SC'11): ten rounds of two 32x32->64
+ * multiplies by the round multipliers, the high halves xored with the other
  * counter words and the key, the key bumped by the Weyl constants between
  * rounds. */
-static void philox4x64_10(const uint64_t ctr[4], const uint64_t key[2], uint64_t out[4]) {
-  const uint64_t M0 = 0xD2E7470EE14C6C93ull, M1 = 0xCA5A826395121157ull;
-  const uint64_t W0 = 0x9E3779B97F4A7C15ull, W1 = 0xBB67AE8584CAA73Bull;
-  uint64_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
-  uint64_t k0 = key[0], k1 = key[1];
+static void philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+  const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+  uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+  uint32_t k0 = key[0], k1 = key[1];
   for (int r = 0; r < 10; ++r) {
-    unsigned __int128 p0 = (unsigned __int128)M0 * x0;
-    unsigned __int128 p1 = (unsigned __int128)M1 * x2;
-    uint64_t hi0 = (uint64_t)(p0 >> 64), lo0 = (uint64_t)p0;
-    uint64_t hi1 = (uint64_t)(p1 >> 64), lo1 = (uint64_t)p1;
+    uint64_t p0 = (uint64_t)M0 * x0;
+    uint64_t p1 = (uint64_t)M1 * x2;
+    uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
     x0 = hi1 ^ x1 ^ k0;
     x1 = lo1;
     x2 = hi0 ^ x3 ^ k1;
@@ -109,18 +111,20 @@ static void philox4x64_10(const uint64_t ctr[4], const uint64_t key[2], uint64_t
   out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
 }
 
-void oracle_philox4x64(const uint64_t* ctr, const uint64_t* key, uint64_t* out) {
-  philox4x64_10(ctr, key, out);
+void oracle_philox4x32(const uint32_t* ctr, const uint32_t* key, uint32_t* out) {
+  philox4x32_10(ctr, key, out);
 }
 
 /* keep_ij of the dropout definition in the header (1 = kept). */
 static int dropout_keep(const oracle_mask* m, int N, int b, int h, int i, int j) {
-  uint64_t ctr[4] = {(uint64_t)(j / 16), (uint64_t)i, (uint64_t)b * N + h, 0};
-  uint64_t key[2] = {m->seed, m->offset};
-  uint64_t w[4];
-  philox4x64_10(ctr, key, w);
-  int f = j % 16;
-  uint64_t u = (w[f / 4] >> (16 * (f % 4))) & 0xFFFFull;
+  uint64_t block = m->offset + (uint64_t)(j / 8);
+  uint64_t bh = (uint64_t)b * N + h;
+  uint32_t ctr[4] = {(uint32_t)block, (uint32_t)(block >> 32), (uint32_t)i, (uint32_t)bh};
+  uint32_t key[2] = {(uint32_t)m->seed, (uint32_t)(m->seed >> 32)};
+  uint32_t w[4];
+  philox4x32_10(ctr, key, w);
+  int f = j % 8;
+  uint32_t u = (w[f / 2] >> (16 * (f % 2))) & 0xFFFFu;
   double t = floor(m->keep_prob * 65536.0 + 0.5);
   return (double)u < t;
 }

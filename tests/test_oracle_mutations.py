@@ -40,8 +40,16 @@ MUTATIONS = {
     "additive_neginf_kept": ("      if (val == -INFINITY) { /* an additive -inf masks the pair */",
                              "      if (0) { /* an additive -inf masks the pair */"),
     "philox_round_order": ("    x0 = hi1 ^ x1 ^ k0;", "    x0 = hi0 ^ x1 ^ k0;"),
-    "dropout_counter_transposed": ("  uint64_t ctr[4] = {(uint64_t)(j / 16), (uint64_t)i, (uint64_t)b * N + h, 0};",
-                                   "  uint64_t ctr[4] = {(uint64_t)(i / 16), (uint64_t)j, (uint64_t)b * N + h, 0};"),
+    "dropout_counter_transposed": ("  uint32_t ctr[4] = {(uint32_t)block, (uint32_t)(block >> 32), (uint32_t)i, (uint32_t)bh};",
+                                   "  uint32_t ctr[4] = {(uint32_t)block, (uint32_t)(block >> 32), (uint32_t)bh, (uint32_t)i};"),
+    "dropout_block_of_16_keys": ("  uint64_t block = m->offset + (uint64_t)(j / 8);",
+                                 "  uint64_t block = m->offset + (uint64_t)(j / 16);"),
+    "dropout_key_halves_swapped": ("  uint32_t key[2] = {(uint32_t)m->seed, (uint32_t)(m->seed >> 32)};",
+                                   "  uint32_t key[2] = {(uint32_t)(m->seed >> 32), (uint32_t)m->seed};"),
+    "dropout_field_order": ("  uint32_t u = (w[f / 2] >> (16 * (f % 2))) & 0xFFFFu;",
+                            "  uint32_t u = (w[f % 4] >> (16 * (f / 4))) & 0xFFFFu;"),
+    "philox_weyl_constant": ("  const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;",
+                             "  const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE87u;"),
     "dropout_no_rescale": ("(dropout_keep(m, N, b, h, i, j) ? 1.0 / m->keep_prob : 0.0)",
                            "(dropout_keep(m, N, b, h, i, j) ? 1.0 : 0.0)"),
     "dropout_dp_unmasked": ("        dp *= f[(int64_t)i * Sk + j];", "        dp *= 1.0;"),
@@ -63,8 +71,9 @@ CHECKS = [
     lambda: pins.test_bias_of_zero_and_neginf_equals_the_bool_mask("bool"),
     lambda: pins.test_bias_constant_shift_moves_only_the_lse((2, 3, 6, 9)),
     pins.test_bias_q0_closed_form,
-    pins.test_philox_matches_numpy_bit_generator,
-    pins.test_dropout_mask_layout_matches_numpy_philox,
+    pins.test_philox_known_answer_vectors,
+    pins.test_philox_matches_torch_engine,
+    lambda: pins.test_dropout_mask_layout_matches_torch_philox(77),
     lambda: pins.test_dropout_matches_torch_autograd("causal"),
 ]
 

@@ -539,40 +539,93 @@ def test_bias_bwd_finite_differences(mode):
 
 
 # ---------------------------------------------------------------- dropout (keep_prob < 1)
-# The guide's keep_prob (sec. 3.1/3.2).  The generator is Philox-4x64-10
-# (Salmon et al., SC'11), pinned to numpy's Philox bit generator (a library
-# implementation of the same published algorithm); the mask layout and the
-# dropout arithmetic are pinned to numpy and to torch autograd.
+# The guide's keep_prob (sec. 3.1/3.2).  The generator is Philox-4x32-10
+# (Salmon et al., SC'11), pinned to the published known-answer vectors
+# (tests/golden/philox4x32_10_kat.json) and to torch's header-only Philox
+# engine (ATen/core/PhiloxRNGEngine.h, a library implementation of the same
+# algorithm, compiled here with the host C++ compiler); the mask layout and
+# the dropout arithmetic are pinned to that engine and to torch autograd.
 
-def test_philox_matches_numpy_bit_generator():
+_ENGINE_SRC = r"""
+#include <ATen/core/PhiloxRNGEngine.h>
+#include <cstdio>
+int main() {
+  unsigned long long seed, subsequence, offset;
+  while (std::scanf("%llu %llu %llu", &seed, &subsequence, &offset) == 3) {
+    at::philox_engine e(seed, subsequence, offset);
+    unsigned w0 = e(), w1 = e(), w2 = e(), w3 = e();
+    std::printf("%u %u %u %u\n", w0, w1, w2, w3);
+  }
+  return 0;
+}
+"""
+_engine_exe = []
+
+
+def _torch_philox(triples):
+    """First 128-bit block of torch's Philox stream for each (seed,
+    subsequence, offset): Philox-4x32-10 at key (seed lo, seed hi) and
+    counter (offset lo, offset hi, subsequence lo, subsequence hi)."""
+    import subprocess
+    import tempfile
+    from torch.utils import cpp_extension
+    if not _engine_exe:
+        inc = cpp_extension.include_paths()[0]
+        if not os.path.exists(os.path.join(inc, "ATen", "core", "PhiloxRNGEngine.h")):
+            pytest.skip("torch's Philox engine header is not installed")
+        d = tempfile.mkdtemp(prefix="philox_engine_")
+        src, exe = os.path.join(d, "engine.cpp"), os.path.join(d, "engine")
+        with open(src, "w") as f:
+            f.write(_ENGINE_SRC)
+        subprocess.run(["g++", "-O1", "-std=c++17", "-I", inc, "-o", exe, src], check=True,
+                       capture_output=True)
+        _engine_exe.append(exe)
+    text = "".join(f"{s} {q} {o}\n" for s, q, o in triples)
+    out = subprocess.run([_engine_exe[0]], input=text, capture_output=True, text=True,
+                         check=True).stdout.split()
+    return np.array([int(x) for x in out], dtype=np.uint32).reshape(-1, 4)
+
+
+def test_philox_known_answer_vectors():
+    with open(os.path.join(GOLD, "philox4x32_10_kat.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        words = [int(x, 16) for x in c["counter"]], [int(x, 16) for x in c["key"]]
+        want = np.array([int(x, 16) for x in c["out"]], dtype=np.uint32)
+        np.testing.assert_array_equal(oracle.philox4x32(*words), want)
+
+
+def test_philox_matches_torch_engine():
     rng = np.random.default_rng(160)
-    for _ in range(20):
-        ctr = rng.integers(1, 2**63, size=4, dtype=np.uint64)
-        key = rng.integers(0, 2**63, size=2, dtype=np.uint64) * np.uint64(2) + np.uint64(1)
-        prev = ctr.copy()
-        prev[0] -= np.uint64(1)          # numpy increments the counter before each block
-        want = np.random.Philox(counter=prev, key=key).random_raw(4)
-        np.testing.assert_array_equal(oracle.philox4x64(ctr, key), want)
+    triples, words = [], []
+    for _ in range(40):
+        c = [int(x) for x in rng.integers(0, 2**32, size=4, dtype=np.uint64)]
+        k = [int(x) for x in rng.integers(0, 2**32, size=2, dtype=np.uint64)]
+        triples.append((k[0] | (k[1] << 32), c[2] | (c[3] << 32), c[0] | (c[1] << 32)))
+        words.append((c, k))
+    want = _torch_philox(triples)
+    for (c, k), w in zip(words, want):
+        np.testing.assert_array_equal(oracle.philox4x32(c, k), w)
 
 
-def test_dropout_mask_layout_matches_numpy_philox():
+@pytest.mark.parametrize("offset", [77, 2**64 - 3])
+def test_dropout_mask_layout_matches_torch_philox(offset):
+    """keep(b, h, i, j): 16-bit field j mod 8 of the block offset + j / 8 of
+    torch's Philox stream with that seed and subsequence (b N + h) 2^32 + i;
+    the second offset makes the block index wrap past 2^64."""
     B, N, Sq, Sk = 2, 3, 5, 40
-    keep_prob, seed, offset = 0.6, 0x1234_5678_9ABC_DEF0, 77
+    keep_prob, seed = 0.6, 0x1234_5678_9ABC_DEF0
     keep = oracle.dropout_keep_mask(B, N, Sq, Sk, keep_prob, seed, offset)
     t = math.floor(keep_prob * 65536 + 0.5)
-    for b in range(B):
-        for h in range(N):
-            for i in range(Sq):
-                for jg in range(0, Sk, 16):
-                    # counter (j / 16, i, b*N + h, 0) as a 256-bit integer;
-                    # numpy increments it before producing a block
-                    ctr = (jg // 16) | (i << 64) | ((b * N + h) << 128)
-                    words = np.random.Philox(counter=(ctr - 1) % (1 << 256), key=seed | (offset << 64)
-                                             ).random_raw(4)
-                    for j in range(jg, min(jg + 16, Sk)):
-                        f = j % 16
-                        u = (int(words[f // 4]) >> (16 * (f % 4))) & 0xFFFF
-                        assert keep[b, h, i, j] == (u < t), (b, h, i, j)
+    idx = [(b, h, i, jb) for b in range(B) for h in range(N) for i in range(Sq)
+           for jb in range((Sk + 7) // 8)]
+    blocks = _torch_philox([(seed, ((b * N + h) << 32) | i, (offset + jb) % 2**64)
+                            for b, h, i, jb in idx])
+    for (b, h, i, jb), words in zip(idx, blocks):
+        for j in range(8 * jb, min(8 * jb + 8, Sk)):
+            f = j % 8
+            u = (int(words[f // 2]) >> (16 * (f % 2))) & 0xFFFF
+            assert keep[b, h, i, j] == (u < t), (b, h, i, j)
 
 
 def test_dropout_keep_rate_and_independence():
