@@ -461,25 +461,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           av[e] = (a_in && q0 + e < p.Sq) ? __ldg(acol + int64_t(q0 + e) * p.a_sq) : 0.f;
       }
       // Dropout keep bits of the 64 queries for key j (bit e: query q0 + e).
-      // Philox blocks hold 16 keys of one query, so each lane of a half-warp
-      // (16 consecutive keys) draws the blocks of 4 queries, and a ballot
-      // per key bit transposes them across the half-warp.
+      // Philox blocks hold 8 keys of one query, so each lane of an 8-lane
+      // group (8 consecutive keys) draws the blocks of 8 queries, and a
+      // ballot per key bit transposes them across the group.
       uint32_t kb[2] = {~0u, ~0u};
       if (has_drop) {
-        const int hw = lane >> 4, rr = lane & 15;
-        const int jg = (c.k0 + wq * 32 + hw * 16) >> 4;
+        const int g8 = lane >> 3, rr = lane & 7;
+        const int jb = (c.k0 + wq * 32 + g8 * 8) >> 3;
         const int64_t bh = int64_t(c.b) * p.N + c.h;
         kb[0] = kb[1] = 0u;
 #pragma unroll 1
-        for (int cq = 0; cq < 4; ++cq) {
-          const uint32_t m16 = dropout_bits16(p.seed, p.offset, p.keep_t, jg, q0 + 16 * cq + rr, bh);
+        for (int cq = 0; cq < 8; ++cq) {
+          const uint32_t m8 = dropout_bits8(p.seed, p.offset, p.keep_t, jb, q0 + 8 * cq + rr, bh);
           uint32_t got = 0;
 #pragma unroll
-          for (int f = 0; f < 16; ++f) {
-            const uint32_t bal = __ballot_sync(~0u, (m16 >> f) & 1u);
-            if (f == rr) got = (bal >> (16 * hw)) & 0xFFFFu;
+          for (int f = 0; f < 8; ++f) {
+            const uint32_t bal = __ballot_sync(~0u, (m8 >> f) & 1u);
+            if (f == rr) got = (bal >> (8 * g8)) & 0xFFu;
           }
-          kb[cq >> 1] |= got << (16 * (cq & 1));
+          kb[cq >> 2] |= got << (8 * (cq & 3));
         }
       }
       const bool got_s = mbar_wait_s(BAR(C::bSFull + b), mine & 1, abort_addr);

@@ -827,14 +827,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t pk[16];
           uint32_t pk8[8];  // e4m3: keys 32 q4 .. 32 q4 + 31, four per column
-          // Dropout keep bits of these 32 keys (two Philox blocks of 16).
+          // Dropout keep bits of these 32 keys (four Philox blocks of 8).
           uint32_t kb32 = ~0u;
-          if (has_drop && row_real) {
-            const int jg = (k0 + 32 * q4) >> 4;
-            const int64_t bh = int64_t(c.b) * p.N + c.h;
-            kb32 = dropout_bits16(p.seed, p.offset, p.keep_t, jg, i, bh) |
-                   (dropout_bits16(p.seed, p.offset, p.keep_t, jg + 1, i, bh) << 16);
-          }
+          if (has_drop && row_real)
+            kb32 = dropout_bits32(p.seed, p.offset, p.keep_t, (k0 + 32 * q4) >> 3, i,
+                                  int64_t(c.b) * p.N + c.h);
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
             const uint64_t s2 = f2_pack(__uint_as_float(sr[q4][e]), __uint_as_float(sr[q4][e + 1]));

@@ -99,8 +99,8 @@ __global__ void __launch_bounds__(kSimtWarps * 32)
       const float pj = expf(s - m_use);        // 0 when masked
       // P V takes the kept, rescaled p (philox.cuh); l sums p before dropout
       const float pv = (p.dropout && j < p.Sk && pj != 0.f)
-                           ? (((dropout_bits16(p.seed, p.offset, p.keep_t, j >> 4, i,
-                                               int64_t(b) * p.N + h) >> (j & 15)) & 1u)
+                           ? (((dropout_bits8(p.seed, p.offset, p.keep_t, j >> 3, i,
+                                              int64_t(b) * p.N + h) >> (j & 7)) & 1u)
                                   ? pj * p.inv_keep
                                   : 0.f)
                            : pj;
@@ -213,8 +213,8 @@ __global__ void __launch_bounds__(kBwdWarps * 32)
         pj = expf(s - lse_i);
         float f = 1.f;  // dropout factor keep / keep_prob (philox.cuh)
         if (p.dropout)
-          f = ((dropout_bits16(p.seed, p.offset, p.keep_t, j >> 4, i, int64_t(b) * p.N + h) >>
-                (j & 15)) & 1u) ? p.inv_keep : 0.f;
+          f = ((dropout_bits8(p.seed, p.offset, p.keep_t, j >> 3, i, int64_t(b) * p.N + h) >>
+                (j & 7)) & 1u) ? p.inv_keep : 0.f;
         dsj = pj * (f * dpd - dl_i);
         pj *= f;  // dV takes the kept, rescaled p
       }

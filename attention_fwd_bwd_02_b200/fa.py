@@ -276,7 +276,8 @@ def make_mask(shape: FaShape, *, causal=False, atten_mask=None, padding_kv_len=N
 
 
 def make_dropout(keep_prob, seed, offset) -> Optional[FaDropout]:
-    """The Philox key of the dropout mask (include/fa.h, fa_dropout); None
+    """The Philox seed and block offset of the dropout mask (include/fa.h,
+    fa_dropout); None
     when keep_prob == 1.  keep_prob < 1 needs an explicit seed."""
     if not (0.0 < float(keep_prob) <= 1.0):
         raise FaError(FA_ERR_INVALID_ARG, f"keep_prob {keep_prob} outside (0, 1]")
@@ -356,8 +357,9 @@ def fwd(query, key, value, head_num=None, input_layout="BNSD", pse=None,
     -inf; -inf masks the pair).  causal: the
     lower-triangular rule.  padding_kv_len: int [B] valid keys per batch.
     modality_ids [B, S] with the 2x2 ``allow`` table and ``allow_diag``.
-    keep_prob < 1: dropout with the Philox mask keyed by (seed, offset)
-    (include/fa.h, fa_dropout); pass the same values to bwd.
+    keep_prob < 1: dropout with the Philox mask of seed and offset
+    (include/fa.h, fa_dropout; offset counts 128-bit blocks, so a fresh
+    mask needs offset advanced by ceil(Sk / 8)); pass the same values to bwd.
     float8_e4m3fn q/k/v (D = 128): the fp8 forward; out is bf16, and the
     caller folds the dequantisation factors of q and k into scale and
     multiplies out by that of v.

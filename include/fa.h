@@ -136,10 +136,15 @@ typedef struct {
  * LSE stays that of the probabilities before dropout.  The keep mask is a
  * function of (seed, offset, b, h, i, j) only, so the backward regenerates
  * it exactly: element (b, h, i, j) is kept iff u < round(keep_prob * 65536)
- * for u the 16-bit field j mod 16 (word (j mod 16) / 4, bits 16 * (j mod 4))
- * of Philox-4x64-10 (Salmon et al., SC'11) at counter (j / 16, i, b*N + h, 0)
- * and key (seed, offset).  Pass the same (seed, offset) to fa_bwd; advance
- * `offset` (or change `seed`) between calls for fresh masks. */
+ * for u the 16-bit field j mod 8 (word (j mod 8) / 2, bits 16 * (j mod 2))
+ * of Philox-4x32-10 (Salmon et al., SC'11) with key (seed mod 2^32,
+ * seed / 2^32) and counter (c0, c1) = offset + j / 8 (mod 2^64), c2 = i,
+ * c3 = (b*N + h) mod 2^32.  That is block offset + j / 8 of the Philox
+ * stream with this seed and subsequence (b*N + h) * 2^32 + i, the
+ * convention of torch's Philox engine: `offset` counts 128-bit blocks, and a
+ * call reads blocks offset .. offset + ceil(Sk / 8) - 1 of each stream.
+ * Pass the same (seed, offset) to fa_bwd; for a fresh mask advance `offset`
+ * by at least ceil(Sk / 8), or change `seed`. */
 typedef struct {
   uint64_t seed;
   uint64_t offset;

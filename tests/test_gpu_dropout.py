@@ -1,5 +1,5 @@
 """Dropout (keep_prob < 1, the FlashAttentionScore guide's keep_prob) on the
-GPU against the fp64 oracle: the same Philox-4x64-10 mask (include/fa.h,
+GPU against the fp64 oracle: the same Philox-4x32-10 mask (include/fa.h,
 fa_dropout) must come out of the forward and the backward kernels, bit for
 bit, and the outputs and gradients must match the oracle's.  Needs a B200
 (sm_100a).
