@@ -108,6 +108,8 @@ fa_status make_problem(const fa_shape* s, const fa_pse* pse, const fa_mask* m,
       q.m_sb = m->mask_stride_b;
       q.m_sh = m->mask_stride_h;
       q.m_sq = m->mask_stride_q;
+      q.mask_vec = aligned16(m->mask) && m->mask_stride_b % 16 == 0 &&
+                   m->mask_stride_h % 16 == 0 && m->mask_stride_q % 16 == 0;
       q.tile_map = m->tile_map;
       q.tm_heads = m->mask_stride_h == 0 ? 1 : s->N;
     }

@@ -22,6 +22,7 @@ struct Problem {
   const int32_t* kv_len;
   const uint8_t* mask;
   int64_t m_sb, m_sh, m_sq;
+  uint32_t mask_vec;        // 1: 16-byte aligned bool-mask rows, 16-byte loads allowed
   const uint8_t* tile_map;  // [B][tm_heads][q tiles][k tiles] or null
   int tm_heads;
   const int32_t* ids;       // modality ids [B][Sk]
@@ -85,6 +86,24 @@ __device__ __forceinline__ bool pair_visible(const Problem& p, int b, int h,
 
 // Bits [lo, hi] (inclusive, positions counted from 0) that fall in 32-bit
 // word w of a bit row, i.e. positions 32w .. 32w+31.
+// Bit e (0..3) set iff byte e of x is nonzero: the high bit of each byte of
+// ((x & 0x7f..) + 0x7f..) | x is set iff the byte is nonzero (no carry
+// crosses a byte), and the multiply gathers bits 7, 15, 23, 31 into 21..24.
+__device__ __forceinline__ uint32_t nonzero_bytes4(uint32_t x) {
+  const uint32_t hb = (((x & 0x7F7F7F7Fu) + 0x7F7F7F7Fu) | x) & 0x80808080u;
+  return ((hb >> 7) * 0x00204081u) >> 21 & 0xFu;
+}
+
+// Bit e (0..31) set iff bool-mask byte row[e] is nonzero; row is 16-byte
+// aligned and holds at least 32 bytes.
+__device__ __forceinline__ uint32_t mask_bits32_vec(const uint8_t* row) {
+  const uint4 a = __ldg(reinterpret_cast<const uint4*>(row));
+  const uint4 b = __ldg(reinterpret_cast<const uint4*>(row + 16));
+  return nonzero_bytes4(a.x) | nonzero_bytes4(a.y) << 4 | nonzero_bytes4(a.z) << 8 |
+         nonzero_bytes4(a.w) << 12 | nonzero_bytes4(b.x) << 16 | nonzero_bytes4(b.y) << 20 |
+         nonzero_bytes4(b.z) << 24 | nonzero_bytes4(b.w) << 28;
+}
+
 __device__ __forceinline__ uint32_t range_bits(int lo, int hi, int w) {
   const int a = max(lo - 32 * w, 0), b = min(hi - 32 * w, 31);
   if (a > b) return 0u;

@@ -681,6 +681,24 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (k1 + 32 * m4 < p.Sk) prefetch_l2(an + 32 * m4);
           }
         }
+        // Bool-mask bits of this row's 128 keys, read before S is ready
+        // (16-byte loads when the rows are aligned and the tile is full).
+        uint32_t mb[4] = {~0u, ~0u, ~0u, ~0u};
+        if (mrow && cls == 1) {
+          if (p.mask_vec && k0 + kBN <= p.Sk) {
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) mb[wd] = mask_bits32_vec(mrow + k0 + 32 * wd);
+          } else {
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+              uint32_t m = 0;
+              const int jw = k0 + 32 * wd;
+#pragma unroll 1
+              for (int e = 0; e < 32 && jw + e < p.Sk; ++e) m |= uint32_t(mrow[jw + e] != 0) << e;
+              mb[wd] = m;
+            }
+          }
+        }
         // Every wait is agreed warp-wide before the .sync.aligned TMEM ops.
         const bool got_s = mbar_wait_s(BAR(C::bSFull + t), steps & 1, abort_addr);
         if (!__all_sync(~0u, got_s)) { ok = false; break; }
@@ -771,14 +789,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int wd = 0; wd < 4; ++wd) vb[wd] = range_bits(0, lim, wd);
             if (mrow) {
-#pragma unroll 1
-              for (int wd = 0; wd < 4; ++wd) {
-                uint32_t m = 0;
-                const int jw = k0 + 32 * wd;
-                for (int e = 0; e < 32 && jw + e < p.Sk; ++e)
-                  m |= uint32_t(mrow[jw + e] != 0) << e;
-                vb[wd] &= m;
-              }
+#pragma unroll
+              for (int wd = 0; wd < 4; ++wd) vb[wd] &= mb[wd];
             }
             if (ids) {
 #pragma unroll

@@ -101,6 +101,31 @@ def test_bf16_bool_mask_with_empty_rows(per_head):
     check_fwd(c, atten_mask=mg, tile_map=tm)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_bool_mask_row_reads_vector_and_byte(D):
+    """The forward reads a 16-byte aligned mask row 16 bytes at a time in
+    full key tiles and byte by byte in the ragged last tile or when the rows
+    are not aligned.  Sk = 400 (rows of 400 bytes, aligned) takes both paths;
+    the same mask as a view one byte into a wider buffer (unaligned rows)
+    takes the byte path everywhere and must give the same result bit for bit.
+    Nonzero bytes other than 1 (2, 0x80, 0xff) mean attend as 1 does."""
+    B, N, Sq, Sk = 2, 3, 200, 400
+    c = I.make_case(f"boolvec_D{D}", B, N, Sq, Sk, D, seed=21)
+    g = torch.Generator().manual_seed(22)
+    vals = torch.tensor([0, 1, 2, 0x80, 0xFF], dtype=torch.uint8)
+    m = vals[torch.randint(0, 5, (B, 1, Sq, Sk), generator=g)]
+    m[:, :, 7, :] = 0                      # a row with no visible key
+    m[1, :, :, 128:256] = 0                # a fully masked tile column
+    aligned = m.cuda()
+    wide = torch.zeros(B, 1, Sq, Sk + 16, dtype=torch.uint8, device="cuda")
+    wide[..., 1:Sk + 1] = aligned
+    unaligned = wide[..., 1:Sk + 1]
+    assert unaligned.data_ptr() % 16 == 1 and unaligned.stride(-1) == 1
+    o1, l1 = check_fwd(c, atten_mask=aligned)
+    o2, l2 = P.gpu_fwd(c, atten_mask=unaligned)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
 def test_fp32_config1():
     c = I.config1()
     check_fwd(c)
