@@ -94,3 +94,25 @@ def test_side_inputs_must_be_on_the_device():
     fa.check_side_inputs("cuda:0", pse=None)          # absent inputs are fine
     with pytest.raises(fa.FaError):
         fa.build_modality_mask(torch.zeros(2, 4, dtype=torch.int32))
+
+
+def test_bool_mask_views_pass_through_with_their_strides():
+    # The forward reads aligned mask rows 16 bytes at a time and anything
+    # else byte by byte: the binding must hand both kinds of view over as
+    # they are (pointer and strides), copying only what the kernel cannot
+    # index (a non-unit last stride or a shape to broadcast).
+    shp = fa.FaShape(2, 3, 5, 32, 64, fa.FA_LAYOUT_BNSD, fa.FA_BF16)
+    wide = torch.zeros(2, 1, 5, 48, dtype=torch.uint8)
+    view = wide[..., 1:33]
+    keep = fa._Keep()
+    m = fa.make_mask(shp, atten_mask=view, keep=keep)
+    assert m.mask == view.data_ptr() == wide.data_ptr() + 1
+    assert (m.mask_stride_b, m.mask_stride_h, m.mask_stride_q) == (5 * 48, 0, 48)
+    full = torch.ones(2, 3, 5, 32, dtype=torch.bool)
+    m = fa.make_mask(shp, atten_mask=full, keep=keep)
+    assert m.mask == full.data_ptr()
+    assert (m.mask_stride_b, m.mask_stride_h, m.mask_stride_q) == (3 * 5 * 32, 5 * 32, 32)
+    # a transposed view (last stride != 1) is copied into a contiguous mask
+    t = torch.ones(2, 3, 32, 5, dtype=torch.uint8).transpose(-1, -2)
+    m = fa.make_mask(shp, atten_mask=t, keep=keep)
+    assert m.mask != t.data_ptr() and m.mask_stride_q == 32
