@@ -62,7 +62,7 @@ def test_dense_term_must_be_on_the_device_and_broadcast():
 
 
 @pytest.mark.skipif(not torch.cuda.is_available(), reason="needs CUDA tensors")
-def test_dense_term_shapes_on_device():  # pragma: no cover - exercised on the GPU machine
+def test_dense_term_shapes_on_device():  # pragma: no cover - needs CUDA tensors
     keep = fa._Keep()
     ok = [(5, 7), (1, 3, 5, 7), (2, 1, 5, 7), (2, 3, 5, 7)]
     for shp in ok:
