@@ -96,7 +96,11 @@ typedef struct {
   const int32_t* kv_len;        /* [B] device, FA_MASK_KV_PADDING            */
   const uint8_t* mask;          /* device, FA_MASK_BOOL; element (b,h,i,j) at
                                    b*stride_b + h*stride_h + i*stride_q + j;
-                                   a zero stride broadcasts that axis        */
+                                   a zero stride broadcasts that axis.  With
+                                   the pointer and all strides multiples of
+                                   16 bytes the forward reads rows 16 bytes
+                                   at a time (otherwise byte by byte: the
+                                   same result, slower)                      */
   int64_t mask_stride_b, mask_stride_h, mask_stride_q;
   const uint8_t* tile_map;      /* optional, from fa_build_mask_tile_map for
                                    this very mask and shape: lets the kernels
