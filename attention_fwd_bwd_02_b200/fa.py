@@ -277,8 +277,8 @@ def make_mask(shape: FaShape, *, causal=False, atten_mask=None, padding_kv_len=N
 
 def make_dropout(keep_prob, seed, offset) -> Optional[FaDropout]:
     """The Philox seed and block offset of the dropout mask (include/fa.h,
-    fa_dropout); None
-    when keep_prob == 1.  keep_prob < 1 needs an explicit seed."""
+    fa_dropout); None when keep_prob == 1.  keep_prob < 1 needs an explicit
+    seed."""
     if not (0.0 < float(keep_prob) <= 1.0):
         raise FaError(FA_ERR_INVALID_ARG, f"keep_prob {keep_prob} outside (0, 1]")
     if float(keep_prob) == 1.0:
