@@ -682,6 +682,40 @@ def test_dropout_matches_torch_autograd(mode):
     np.testing.assert_allclose(dv, vt.grad.numpy(), atol=1e-12, rtol=0)
 
 
+@pytest.mark.parametrize("mode", ["causal", "bool", "modality"])
+def test_all_terms_together_match_torch_autograd(mode):
+    """A dense additive term, ALiBi, a mask and dropout at once: the scaled
+    scores plus ALiBi plus the term are masked, softmaxed, dropped and
+    rescaled, then multiply V (guide sec. 2 and sec. 4 step 1, with the
+    keep_prob of sec. 3.2); LSE is that of the scores before dropout."""
+    B, N, S, D = 2, 3, 11, 4
+    keep_prob, seed, offset = 0.6, 77, 5
+    gen = torch.Generator().manual_seed(185)
+    q, k, v, do = (torch.randn(B, N, S, D, dtype=torch.float64, generator=gen) for _ in range(4))
+    bias = torch.randn(B, N, S, S, dtype=torch.float64, generator=gen)
+    slopes = np.array([0.5, 0.25, 0.125])
+    kw = _mask_kwargs(mode, B, N, S, S, seed=186)
+    allowed = _allowed_dense(mode, B, N, S, S, kw)
+    keep = torch.as_tensor(oracle.dropout_keep_mask(B, N, S, S, keep_prob, seed, offset)).bool()
+    i = torch.arange(S, dtype=torch.float64)
+    alibi = -torch.as_tensor(slopes)[:, None, None] * (i[:, None] - i[None, :]).abs()
+    qt, kt, vt = (t.clone().requires_grad_(True) for t in (q, k, v))
+    s = (qt @ kt.transpose(-1, -2)) * 0.4 + alibi + bias
+    p = torch.softmax(s.masked_fill(~allowed, float("-inf")), -1)
+    p = torch.nan_to_num(p, nan=0.0)   # rows with no allowed key give 0
+    ref = (p * keep / keep_prob) @ vt
+    (ref * do).sum().backward()
+    okw = dict(kw, slopes=slopes, bias=bias.numpy(), dropout=(keep_prob, seed, offset))
+    out, lse = oracle.fwd(q, k, v, 0.4, **okw)
+    np.testing.assert_allclose(out, ref.detach().numpy(), atol=1e-12, rtol=0)
+    ref_lse = torch.logsumexp(s.detach().masked_fill(~allowed, float("-inf")), -1).numpy()
+    np.testing.assert_allclose(lse, ref_lse, atol=1e-12, rtol=0)
+    dq, dk, dv = oracle.bwd(q, k, v, do, 0.4, **okw)
+    np.testing.assert_allclose(dq, qt.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dk, kt.grad.numpy(), atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dv, vt.grad.numpy(), atol=1e-12, rtol=0)
+
+
 def test_dropout_bwd_finite_differences():
     B, N, S, D = 1, 2, 5, 3
     q, k, v, do = (_rand((B, N, S, D), 190 + n) for n in range(4))
