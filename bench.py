@@ -628,7 +628,9 @@ def run_variant(args):
     S=2048 D=128) and prints one JSON line (not the main line):
       e4m3    -- the fp8 forward (fa_fwd with e4m3 q, k, v; bf16 out);
       dense   -- fa_fwd + fa_bwd with a dense [1, N, S, S] fp32 term;
-      dropout -- fa_fwd + fa_bwd with keep_prob = 0.9."""
+      dropout -- fa_fwd + fa_bwd with keep_prob = 0.9;
+      mask    -- fa_fwd + fa_bwd with a random [B, 1, S, S] bool mask (half
+                 the pairs) on top of the causal rule, no tile map."""
     import torch
     from attention_fwd_bwd_02_b200 import fa
     from attention_fwd_bwd_02_b200 import inputs as I
@@ -645,6 +647,9 @@ def run_variant(args):
     elif args.variant == "dense":
         g = torch.Generator(device=dev).manual_seed(3)
         kw["pse"] = torch.randn(1, N, S, S, device=dev, generator=g)
+    elif args.variant == "mask":
+        g = torch.Generator(device=dev).manual_seed(4)
+        kw["atten_mask"] = (torch.rand(B, 1, S, S, device=dev, generator=g) < 0.5).to(torch.uint8)
     else:
         kw.update(keep_prob=0.9, seed=1234, offset=0)
     out, lse = fa.fwd(q, k, v, N, **kw)
@@ -700,9 +705,10 @@ def main():
     ap.add_argument("--configs", action="store_true",
                     help="instead of the main line, time every workload of the "
                          "source pages (one JSON line each)")
-    ap.add_argument("--variant", choices=["e4m3", "dense", "dropout"],
+    ap.add_argument("--variant", choices=["e4m3", "dense", "dropout", "mask"],
                     help="instead of the main line, time one variant of the "
-                         "headline workload (fp8 forward, dense term, dropout)")
+                         "headline workload (fp8 forward, dense term, dropout, "
+                         "bool mask)")
     args = ap.parse_args()
     if args.impl == "ours":
         args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
